@@ -1,0 +1,132 @@
+"""Float64 CPU oracle of the LSA decode step (FlashMemory-DeepSeek-V4).
+
+TEST INFRASTRUCTURE ONLY: the test suite, the package smoke check and the
+benchmark's CPU-baseline leg may import this package; the product path never
+does. It shares no code with the CUDA path. The arithmetic lives in plain C
+(``lsa_oracle.c``, float64, loops in the order the definitions give); this file
+only widens inputs to float64 and loops over the sequences of a batch.
+
+What it computes, per sequence (review of FlashMemory-DeepSeek-V4 on
+dimensionstp.github.io, section 3-2 (2)-(3); arXiv abstract):
+
+1. chunk scores  s_i = max_j <q_emb[j], chunk_emb[i]>   (dual-encoder inner product;
+   the max over the 64 lookahead queries, as the per-layer ensemble is a max);
+2. top-k keep mask: order by (score desc, index asc), keep k, report ascending;
+3. gather: the kept chunks' K/V rows, in kept order (a compaction);
+4. exact softmax attention of the decode query over the kept tokens only,
+   scale 1/sqrt(Dh), returning the output and the log-sum-exp per head;
+5. footprint = k * chunk_len / L.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(hand-worked fixtures in ``tests/golden/``, closed forms, a brute-force
+characterisation of top-k, and torch's float64 scaled-dot-product attention
+as an independent library reference).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        i64, dp, ip = ctypes.c_int64, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int32)
+        lib.lsa_oracle_chunk_scores.argtypes = [i64, i64, i64, dp, dp, dp]
+        lib.lsa_oracle_chunk_scores.restype = None
+        lib.lsa_oracle_topk.argtypes = [i64, dp, i64, ip]
+        lib.lsa_oracle_topk.restype = ctypes.c_int
+        lib.lsa_oracle_attention.argtypes = [i64, i64, i64, ctypes.c_double, dp, dp, dp, dp, dp, dp]
+        lib.lsa_oracle_attention.restype = None
+        lib.lsa_oracle_footprint.argtypes = [i64, i64, i64]
+        lib.lsa_oracle_footprint.restype = ctypes.c_double
+        _lib = lib
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _dp(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def chunk_scores(q_emb, chunk_emb) -> np.ndarray:
+    """s[i] = max_j sum_d q_emb[j, d] * chunk_emb[i, d]   (q_emb [Q, E] or [E]; chunk_emb [n, E])."""
+    q = _f64(q_emb)
+    if q.ndim == 1:
+        q = q[None, :]
+    e = _f64(chunk_emb)
+    n, E = e.shape
+    assert q.shape[1] == E
+    s = np.empty(n, dtype=np.float64)
+    _load().lsa_oracle_chunk_scores(n, q.shape[0], E, _dp(q), _dp(e), _dp(s))
+    return s
+
+
+def topk(scores, k: int) -> np.ndarray:
+    """Kept chunk indices (int32, ascending): the k best by (score desc, index asc)."""
+    s = _f64(scores)
+    ids = np.empty(max(int(k), 0), dtype=np.int32)
+    rc = _load().lsa_oracle_topk(s.shape[0], _dp(s), int(k),
+                                 ids.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
+    if rc != 0:
+        raise ValueError("top-k rejected its input (non-finite score, or k outside 1..n)")
+    return ids
+
+
+def attention(q, K, V, scale: float | None = None):
+    """Exact softmax attention of one decode query. q [H, Dh]; K, V [T, H, Dh].
+
+    Returns (out [H, Dh], lse [H]) in float64; scale defaults to 1/sqrt(Dh)."""
+    q, K, V = _f64(q), _f64(K), _f64(V)
+    T, H, Dh = K.shape
+    assert q.shape == (H, Dh) and V.shape == K.shape and T >= 1
+    if scale is None:
+        scale = 1.0 / math.sqrt(Dh)
+    out = np.empty((H, Dh), dtype=np.float64)
+    lse = np.empty(H, dtype=np.float64)
+    z = np.empty(T, dtype=np.float64)
+    _load().lsa_oracle_attention(T, H, Dh, float(scale), _dp(q), _dp(K), _dp(V),
+                                 _dp(out), _dp(lse), _dp(z))
+    return out, lse
+
+
+def kept_tokens(ids, chunk_len: int) -> np.ndarray:
+    """Token positions (within the sequence) covered by the kept chunks, in kept order."""
+    ids = np.asarray(ids, dtype=np.int64)
+    return (ids[:, None] * chunk_len + np.arange(chunk_len)[None, :]).reshape(-1)
+
+
+def gather(cache, ids, chunk_len: int) -> np.ndarray:
+    """Resident buffer of one sequence: row j*C + t is row ids[j]*C + t of ``cache`` [L, ...]."""
+    return np.asarray(cache)[kept_tokens(ids, chunk_len)]
+
+
+def footprint(k: int, chunk_len: int, context_len: int) -> float:
+    """Resident KV footprint: k * chunk_len / L."""
+    return _load().lsa_oracle_footprint(int(k), int(chunk_len), int(context_len))
+
+
+def decode_step(q_emb, chunk_emb, q, K, V, k: int, chunk_len: int, scale: float | None = None):
+    """One sequence's full step: scores -> top-k -> gather -> attention.
+
+    K and V are the full caches [L, H, Dh] of the sequence (or callables that
+    return the rows of given token positions). Returns (ids, out, lse, scores)."""
+    s = chunk_scores(q_emb, chunk_emb)
+    ids = topk(s, k)
+    tok = kept_tokens(ids, chunk_len)
+    Kk = K(tok) if callable(K) else np.asarray(K)[tok]
+    Vk = V(tok) if callable(V) else np.asarray(V)[tok]
+    out, lse = attention(q, Kk, Vk, scale)
+    return ids, out, lse, s

@@ -1,0 +1,69 @@
+"""Host-side checks of the seeded input generator (datagen)."""
+import numpy as np
+import torch
+
+import datagen
+
+
+def test_splitmix64_known_answers():
+    # SplitMix64 seeded with 0: the first three outputs of the published generator
+    key = np.array([0], dtype=np.uint64)
+    n = np.arange(1, 4, dtype=np.uint64)
+    got = datagen.mix64(key + n * datagen.GAMMA)
+    assert [int(v) for v in got] == [0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4, 0x06C45D188009454F]
+
+
+def test_normal_statistics_and_exactness():
+    x = datagen.normal_f32(123, 4, np.arange(400_000))
+    assert abs(float(x.mean())) < 0.01
+    assert abs(float(x.var()) - 1.0) < 0.01
+    assert float(np.abs(x).max()) < 6.0
+    # every value is an integer multiple of 2**-16 (exact in float32)
+    r = x.astype(np.float64) * 65536.0
+    np.testing.assert_array_equal(r, np.round(r))
+
+
+def test_normal_is_counter_based():
+    a = datagen.normal_f32(5, 4, np.arange(1000))
+    b = datagen.normal_f32(5, 4, np.arange(500, 1000))
+    np.testing.assert_array_equal(a[500:], b)
+    c = datagen.normal_f32(6, 4, np.arange(1000))
+    assert not np.array_equal(a, c)
+
+
+def test_bf16_rounding_matches_torch():
+    x = np.concatenate([datagen.normal_f32(1, 1, np.arange(100_000)) * np.float32(37.0),
+                        np.array([1.00390625, 1.01171875, -1.00390625, 0.0, -0.0], np.float32)])
+    ours = datagen.bf16_bits(x)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(ours, ref)
+    np.testing.assert_array_equal(datagen.bf16_to_f32(ours),
+                                  torch.from_numpy(x).to(torch.bfloat16).float().numpy())
+
+
+def test_workload_shapes():
+    for name in datagen.WORKLOADS:
+        w = datagen.workload(name)
+        assert len(w.N) == w.B and len(w.k) == w.B
+        assert all(1 <= k <= n for k, n in zip(w.k, w.N))
+    w = datagen.workload("mixed")
+    assert w.B == 32 and not w.uniform
+    assert all(32768 <= l <= 524288 and l % 64 == 0 for l in w.L)
+    assert all(k == int(np.floor(0.135 * n + 0.5)) for k, n in zip(w.k, w.N))
+    assert datagen.workload("500k").k[0] == 819 and datagen.workload("1m").k[0] == 2212
+
+
+def test_kv_rows_layout():
+    w = datagen.small_workload()
+    r = datagen.kv_rows(w, "K", [3, 0], [1])
+    idx = (np.array([3, 0])[:, None] * w.H + 1) * w.Dh + np.arange(w.Dh)[None, :]
+    np.testing.assert_array_equal(r[:, 0, :], datagen.normal_f32(w.seed, 4, idx))
+
+
+def test_make_inputs_tiny_planting():
+    w = datagen.workload("tiny")
+    x = datagen.make_inputs(w)
+    assert x["q_emb"].shape == (1, 1, 128) and x["chunk_emb"].shape == (64, 128)
+    pos = datagen.planted_positions(w, 0)
+    d = x["chunk_emb"][pos] - x["q_emb"][0, 0][None, :]
+    assert float(np.abs(d).max()) < 0.1 * 6.0 + 1e-6

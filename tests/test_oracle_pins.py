@@ -1,0 +1,256 @@
+"""Pins for the float64 oracle: hand-worked fixtures, closed forms, brute force
+and an independent library routine. Each test would fail for a plausible slip
+in the oracle (dropped term, wrong sign or index, transposed operand, wrong
+tie rule, unkept tokens leaking into the softmax)."""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import datagen
+import oracle
+from tests._golden import load
+
+
+# ---------------------------------------------------------------- scores
+def test_scores_golden_one_query():
+    g = load("scores_tiny.txt")
+    np.testing.assert_array_equal(oracle.chunk_scores(g["q1"], g["emb"]), g["s1"])
+
+
+def test_scores_golden_two_queries_max():
+    g = load("scores_tiny.txt")
+    np.testing.assert_array_equal(oracle.chunk_scores(g["q2"], g["emb"]), g["s2"])
+
+
+def test_scores_unit_vectors_pick_coordinates():
+    # chunk i is the unit vector along axis d_i, so its score is q[d_i]
+    rng = np.random.default_rng(0)
+    E = 16
+    q = rng.standard_normal(E)
+    d = rng.permutation(E)[:10]
+    emb = np.eye(E)[d]
+    np.testing.assert_array_equal(oracle.chunk_scores(q, emb), q[d])
+
+
+def test_scores_exact_on_integers():
+    # integer inputs: the float64 result is exact; int64 matmul is an independent exact reference
+    rng = np.random.default_rng(1)
+    for Q in (1, 3, 64):
+        q = rng.integers(-20, 21, size=(Q, 48))
+        e = rng.integers(-20, 21, size=(37, 48))
+        ref = (e @ q.T).max(axis=1).astype(np.float64)
+        np.testing.assert_array_equal(oracle.chunk_scores(q, e), ref)
+
+
+def test_scores_negative_and_mixed_sign():
+    q = np.array([[-1.0, 0.0], [0.0, -1.0]])
+    e = np.array([[2.0, 3.0], [-4.0, -1.0]])
+    # chunk 0: max(-2, -3) = -2 ; chunk 1: max(4, 1) = 4
+    np.testing.assert_array_equal(oracle.chunk_scores(q, e), [-2.0, 4.0])
+
+
+# ---------------------------------------------------------------- top-k
+@pytest.mark.parametrize("k", [1, 2, 4, 6, 7, 8])
+def test_topk_golden_ties(k):
+    g = load("topk_ties.txt")
+    ids = oracle.topk(g["scores"], int(g[f"k{k}"]))
+    np.testing.assert_array_equal(ids, np.atleast_1d(g[f"ids{k}"]).astype(np.int32))
+
+
+def _valid_topk_sets(s, k):
+    """All k-subsets S with: for i in S, j not in S, s_i > s_j or (s_i == s_j and i < j)."""
+    n = len(s)
+    out = []
+    for S in itertools.combinations(range(n), k):
+        inS = set(S)
+        ok = all((s[i] > s[j]) or (s[i] == s[j] and i < j)
+                 for i in S for j in range(n) if j not in inS)
+        if ok:
+            out.append(list(S))
+    return out
+
+
+def test_topk_brute_force_characterisation():
+    rng = np.random.default_rng(2)
+    for trial in range(300):
+        n = int(rng.integers(1, 11))
+        s = rng.integers(-3, 4, size=n).astype(np.float64)  # many ties
+        k = int(rng.integers(1, n + 1))
+        valid = _valid_topk_sets(s, k)
+        assert len(valid) == 1, (s, k, valid)
+        np.testing.assert_array_equal(oracle.topk(s, k), valid[0])
+
+
+def test_topk_rejects_bad_input():
+    with pytest.raises(ValueError):
+        oracle.topk([1.0, float("nan"), 2.0], 1)
+    with pytest.raises(ValueError):
+        oracle.topk([1.0, float("inf")], 1)
+    with pytest.raises(ValueError):
+        oracle.topk([1.0, 2.0], 0)
+    with pytest.raises(ValueError):
+        oracle.topk([1.0, 2.0], 3)
+
+
+def test_topk_permutation_equivariance_and_scale_invariance():
+    rng = np.random.default_rng(3)
+    s = rng.standard_normal(200)  # distinct almost surely
+    k = 17
+    ids = oracle.topk(s, k)
+    perm = rng.permutation(200)           # new position p holds old chunk perm[p]
+    ids_p = oracle.topk(s[perm], k)
+    np.testing.assert_array_equal(np.sort(perm[ids_p]), ids)
+    np.testing.assert_array_equal(oracle.topk(3.5 * s, k), ids)
+
+
+def test_topk_keeps_the_largest():
+    s = np.array([0.5, -1.0, 9.0, 2.0, 8.0, 3.0])
+    np.testing.assert_array_equal(oracle.topk(s, 3), [2, 4, 5])
+    np.testing.assert_array_equal(oracle.topk(-s, 2), [0, 1])  # sign matters: the two smallest of s
+
+
+# ---------------------------------------------------------------- attention
+def test_attention_golden_two_tokens():
+    g = load("attention_two_tokens.txt")
+    out, lse = oracle.attention(g["q"][None, :], g["K"][:, None, :], g["V"][:, None, :])
+    np.testing.assert_allclose(out[0], g["out"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse[0], g["lse"], rtol=0, atol=1e-15)
+
+
+def _sdpa(q, K, V, mask=None):
+    """torch float64 scaled_dot_product_attention (an independent library routine)."""
+    qt = torch.from_numpy(np.asarray(q, np.float64))[:, None, :]          # [H, 1, Dh]
+    Kt = torch.from_numpy(np.asarray(K, np.float64)).permute(1, 0, 2)     # [H, T, Dh]
+    Vt = torch.from_numpy(np.asarray(V, np.float64)).permute(1, 0, 2)
+    m = None if mask is None else torch.from_numpy(mask)[None, None, :].expand(qt.shape[0], 1, -1)
+    o = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt, attn_mask=m)
+    return o[:, 0, :].numpy()
+
+
+def test_attention_dense_matches_library_sdpa():
+    rng = np.random.default_rng(4)
+    T, H, Dh = 300, 4, 128
+    q, K, V = rng.standard_normal((H, Dh)), rng.standard_normal((T, H, Dh)), rng.standard_normal((T, H, Dh))
+    out, _ = oracle.attention(q, K, V)
+    np.testing.assert_allclose(out, _sdpa(q, K, V), rtol=0, atol=1e-13)
+
+
+def test_sparse_attention_equals_masked_dense():
+    # attention over the kept chunks == dense attention with every unkept token masked out
+    rng = np.random.default_rng(5)
+    n, C, H, Dh, k = 12, 8, 2, 128, 4
+    L = n * C
+    q, K, V = rng.standard_normal((H, Dh)), rng.standard_normal((L, H, Dh)), rng.standard_normal((L, H, Dh))
+    ids = np.sort(rng.permutation(n)[:k]).astype(np.int32)
+    out, _ = oracle.attention(q, oracle.gather(K, ids, C), oracle.gather(V, ids, C))
+    mask = np.zeros(L, dtype=bool)
+    mask[oracle.kept_tokens(ids, C)] = True
+    np.testing.assert_allclose(out, _sdpa(q, K, V, mask), rtol=0, atol=1e-13)
+
+
+def test_attention_single_token_returns_v():
+    rng = np.random.default_rng(6)
+    q, K, V = rng.standard_normal((3, 128)), rng.standard_normal((1, 3, 128)), rng.standard_normal((1, 3, 128))
+    out, lse = oracle.attention(q, K, V)
+    np.testing.assert_allclose(out, V[0], rtol=0, atol=1e-15)
+    z = np.einsum("hd,hd->h", q, K[0]) / math.sqrt(128)
+    np.testing.assert_allclose(lse, z, rtol=0, atol=1e-13)
+
+
+def test_attention_equal_keys_average_values():
+    rng = np.random.default_rng(7)
+    T, H, Dh = 50, 2, 128
+    q = rng.standard_normal((H, Dh))
+    K = np.broadcast_to(rng.standard_normal((1, H, Dh)), (T, H, Dh)).copy()
+    V = rng.standard_normal((T, H, Dh))
+    out, lse = oracle.attention(q, K, V)
+    np.testing.assert_allclose(out, V.mean(axis=0), rtol=0, atol=1e-13)
+    z = np.einsum("hd,hd->h", q, K[0]) / math.sqrt(Dh)
+    np.testing.assert_allclose(lse, z + math.log(T), rtol=0, atol=1e-12)
+
+
+def test_attention_weights_sum_to_one():
+    rng = np.random.default_rng(8)
+    T, H, Dh = 77, 3, 128
+    q, K, V = 3 * rng.standard_normal((H, Dh)), rng.standard_normal((T, H, Dh)), rng.standard_normal((T, H, Dh))
+    _, lse = oracle.attention(q, K, V)
+    z = np.einsum("hd,thd->th", q, K) / math.sqrt(Dh)     # independent score computation
+    np.testing.assert_allclose(np.exp(z - lse[None, :]).sum(axis=0), 1.0, rtol=0, atol=1e-12)
+
+
+def test_attention_scale_is_one_over_sqrt_dh():
+    # with scale = 1/sqrt(Dh) by default, doubling Dh-normalised logits must match an explicit scale
+    rng = np.random.default_rng(9)
+    q, K, V = rng.standard_normal((1, 128)), rng.standard_normal((9, 1, 128)), rng.standard_normal((9, 1, 128))
+    a, _ = oracle.attention(q, K, V)
+    b, _ = oracle.attention(q, K, V, scale=1.0 / math.sqrt(128.0))
+    c, _ = oracle.attention(q / math.sqrt(128.0), K, V, scale=1.0)
+    np.testing.assert_array_equal(a, b)
+    np.testing.assert_allclose(a, c, rtol=0, atol=1e-14)
+
+
+# ---------------------------------------------------------------- gather + whole step
+def test_gather_identity_and_order():
+    L, C = 24, 4
+    K = np.arange(L * 2 * 3, dtype=np.float64).reshape(L, 2, 3)
+    np.testing.assert_array_equal(oracle.gather(K, np.arange(L // C), C), K)
+    g = oracle.gather(K, np.array([5, 1]), C)
+    np.testing.assert_array_equal(g[:C], K[20:24])
+    np.testing.assert_array_equal(g[C:], K[4:8])
+
+
+def test_decode_step_golden():
+    g = load("decode_step_tiny.txt")
+    K = g["K"][:, None, :]
+    V = g["V"][:, None, :]
+    ids, out, lse, s = oracle.decode_step(g["q_emb"], g["emb"], g["q"][None, :], K, V, int(g["k"]), 2)
+    np.testing.assert_array_equal(s, g["scores"])
+    np.testing.assert_array_equal(ids, g["ids"])
+    np.testing.assert_allclose(out[0], g["out"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse[0], g["lse"], rtol=0, atol=1e-15)
+    assert oracle.footprint(int(g["k"]), 2, 8) == g["footprint"]
+
+
+def test_full_keep_equals_dense_attention():
+    # k = every chunk: the LSA step reduces to ordinary dense decode attention
+    rng = np.random.default_rng(10)
+    n, C, E, H, Dh = 6, 4, 8, 2, 128
+    L = n * C
+    q_emb, emb = rng.standard_normal(E), rng.standard_normal((n, E))
+    q, K, V = rng.standard_normal((H, Dh)), rng.standard_normal((L, H, Dh)), rng.standard_normal((L, H, Dh))
+    ids, out, _, _ = oracle.decode_step(q_emb, emb, q, K, V, n, C)
+    np.testing.assert_array_equal(ids, np.arange(n))
+    np.testing.assert_allclose(out, _sdpa(q, K, V), rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------- footprint
+@pytest.mark.parametrize("name,expect", [
+    ("tiny", 0.125), ("128k", 0.125), ("500k", 819 / 8192), ("1m", 2212 / 16384)])
+def test_footprint_of_workloads(name, expect):
+    w = datagen.workload(name)
+    assert oracle.footprint(w.k[0], w.C, w.L[0]) == expect
+
+
+def test_footprint_matches_pages_headline():
+    # the pages' average physical footprint is 13.5% of the full context; the 1M workload keeps
+    # round(0.135 * 16384) = 2212 chunks, i.e. 13.50% resident, an 86.5% cut
+    w = datagen.workload("1m")
+    f = oracle.footprint(w.k[0], w.C, w.L[0])
+    assert abs(f - 0.135) < 1e-4
+    # the 500K workload keeps about 10%, the pages' "over 90% reduction at 500K"
+    w = datagen.workload("500k")
+    assert 1.0 - oracle.footprint(w.k[0], w.C, w.L[0]) > 0.90
+
+
+# ---------------------------------------------------------------- planted structure
+def test_planted_chunks_recovered_tiny():
+    w = datagen.workload("tiny")
+    x = datagen.make_inputs(w)
+    s = oracle.chunk_scores(x["q_emb"][0], x["chunk_emb"])
+    ids = oracle.topk(s, w.k[0])
+    planted = datagen.planted_positions(w, 0)
+    assert len(planted) == 4
+    assert set(planted.tolist()) <= set(ids.tolist())
