@@ -1,0 +1,157 @@
+/*
+ * lsa.h - C ABI of the Lookahead Sparse Attention (LSA) decode step, B200 (sm_100a).
+ *
+ * The method (FlashMemory-DeepSeek-V4, "Lightning Index Ultra-Long Context via
+ * Lookahead Sparse Attention", arXiv 2606.09079): at a decode step a dual-encoder
+ * Neural Memory Indexer scores every historical KV chunk against the query side,
+ * a top-k keep mask keeps the query-critical chunks, and decode attention runs
+ * over the kept chunks only. Sources, by page and section:
+ *   [R3-2.1] dimensionstp.github.io review, section 3-2 (1): the KV cache is
+ *            treated as chunk-granular memory (the cache unit is a chunk);
+ *   [R3-2.2] same review, section 3-2 (2) "Neural Memory Indexer": chunk
+ *            relevance scoring; layer scores are combined with a max;
+ *   [R3-2.3] same review, section 3-2 (3) "Lookahead Sparse Attention",
+ *            steps 4-7: score all chunks, top-k keep mask, attend over the kept
+ *            chunks only; the lookahead window is about 64 tokens;
+ *   [ABS]    the arXiv abstract: the indexer is a standard dual encoder (so a
+ *            relevance score is an inner product) and only the query-critical
+ *            KV chunks stay resident in GPU memory.
+ *
+ * Conventions for every call
+ *   - All tensor pointers are DEVICE pointers owned by the caller, 16-byte
+ *     aligned, row-major and contiguous. The library never allocates or frees
+ *     memory and never synchronises, except lsa_get_device_status.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL is the legacy default stream). Calls can be captured in a CUDA graph.
+ *   - Arguments are validated on the host before anything is launched; a bad
+ *     argument returns LSA_ERR_INVALID_ARG / LSA_ERR_UNSUPPORTED / LSA_ERR_WORKSPACE
+ *     and launches nothing. A launch failure returns LSA_ERR_CUDA.
+ *   - Errors found on the device (a non-finite score, a kept chunk id out of
+ *     range, a bounded wait that gave up) set bits of a sticky error word at the
+ *     start of the workspace; the kernels then skip the bad item instead of
+ *     faulting. lsa_get_device_status reads and clears that word.
+ *   - Ragged batches: with chunk_offsets != NULL, sequence b owns chunks
+ *     [chunk_offsets[b], chunk_offsets[b+1]) of the flattened chunk axis and
+ *     tokens [chunk_offsets[b]*C, chunk_offsets[b+1]*C) of the K/V caches.
+ *     Kept ids are laid out flat: sequence b's k_b ids start at sum_{b'<b} k_b'.
+ */
+#ifndef LSA_H_
+#define LSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define LSA_API __attribute__((visibility("default")))
+#else
+#define LSA_API
+#endif
+
+#define LSA_ABI_VERSION 1
+#define LSA_MAX_BATCH 256   /* sequences per call */
+#define LSA_HEAD_DIM 128    /* Dh: the pages' HEAD_DIM (review, section 4-3) */
+
+typedef enum {
+    LSA_OK = 0,
+    LSA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, k outside 1..N_b */
+    LSA_ERR_WORKSPACE = 2,    /* workspace smaller than lsa_workspace_size() */
+    LSA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+    LSA_ERR_NONFINITE = 4,    /* device: a chunk score was NaN or +-Inf */
+    LSA_ERR_TIMEOUT = 5,      /* device: a bounded wait gave up */
+    LSA_ERR_UNSUPPORTED = 6,  /* a shape this build does not implement */
+    LSA_ERR_BAD_ID = 7        /* device: a kept chunk id was outside 0..N_b-1 */
+} lsa_status;
+
+typedef enum { LSA_F32 = 0, LSA_BF16 = 1 } lsa_dtype;
+
+/* Problem shape of one call. Host memory; copied by value into the launch. */
+typedef struct {
+    int32_t B;          /* sequences, 1..LSA_MAX_BATCH */
+    int32_t Q;          /* query embeddings per sequence: 1 (decode query) .. 256 (64 = lookahead window) */
+    int32_t E;          /* embedding dim; E*sizeof(emb) a power of two in 16..512 bytes, or a multiple of 512 */
+    int32_t H;          /* attention heads (query heads = KV heads), a power of two, 1..128 */
+    int32_t Dh;         /* head dim, must be LSA_HEAD_DIM */
+    int32_t chunk_len;  /* C, tokens per chunk, a power of two, 8..1024 (64 in the workloads) */
+    int32_t N;          /* chunks per sequence when chunk_offsets == NULL */
+    int32_t k;          /* kept chunks per sequence when k_per_seq == NULL */
+    const int64_t *chunk_offsets; /* host [B+1], nondecreasing from 0, or NULL (uniform N) */
+    const int32_t *k_per_seq;     /* host [B], or NULL (uniform k) */
+    lsa_dtype emb_dtype;          /* q_emb and chunk_emb */
+    lsa_dtype kv_dtype;           /* q, K, V, K_res, V_res */
+} lsa_dims;
+
+/* ABI version of the loaded library (LSA_ABI_VERSION). */
+LSA_API int lsa_abi_version(void);
+
+/* Human-readable name of a status code (static string). */
+LSA_API const char *lsa_status_string(lsa_status s);
+
+/* Bytes of device workspace the calls below need for `dims` on the current
+ * device (it depends on the SM count). Writes *bytes; no launch. */
+LSA_API lsa_status lsa_workspace_size(const lsa_dims *dims, size_t *bytes);
+
+/* Clear the workspace's sticky error word (cudaMemsetAsync of its header).
+ * Call once after allocating a workspace. */
+LSA_API lsa_status lsa_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/* Chunk relevance [R3-2.2, ABS, R3-2.3 step 4].
+ *   q_emb     [B][Q][E]      emb_dtype
+ *   chunk_emb [sum N_b][E]   emb_dtype
+ *   scores    [sum N_b]      float32, out:  scores[i] = max_j <q_emb[b][j], chunk_emb[i]>
+ * fp32 accumulation. Q == 1 streams the embeddings on CUDA cores; Q > 1 with bf16
+ * embeddings and E <= 256 runs a tcgen05 tensor-core GEMM with a per-row max. */
+LSA_API lsa_status lsa_score_chunks(const lsa_dims *dims, const void *q_emb, const void *chunk_emb,
+                            float *scores, void *ws, size_t ws_bytes, void *stream);
+
+/* Top-k keep mask [R3-2.3 step 5].
+ *   scores    [sum N_b]   float32
+ *   chunk_ids [sum k_b]   int32, out: per sequence the k_b chunk indices (0..N_b-1,
+ *                         local to the sequence) with the highest scores, ties to the
+ *                         lower index, written in ascending order. -0.0 == +0.0.
+ * A NaN/Inf score sets LSA_ERR_NONFINITE in the sticky word (ids stay in range). */
+LSA_API lsa_status lsa_topk_select(const lsa_dims *dims, const float *scores, int32_t *chunk_ids,
+                           void *ws, size_t ws_bytes, void *stream);
+
+/* Gather of the kept chunks into a compact resident buffer [R3-2.3 step 6, ABS].
+ *   K, V         [sum L_b][H][Dh]   kv_dtype (L_b = N_b * C)
+ *   chunk_ids    [sum k_b]          int32, local chunk indices
+ *   K_res, V_res [sum k_b * C][H][Dh] kv_dtype, out: row j*C+t of sequence b's
+ *                block is row ids[j]*C+t of its cache.
+ * An id outside 0..N_b-1 sets LSA_ERR_BAD_ID and that chunk is left unwritten. */
+LSA_API lsa_status lsa_gather_kv(const lsa_dims *dims, const void *K, const void *V,
+                         const int32_t *chunk_ids, void *K_res, void *V_res,
+                         void *ws, size_t ws_bytes, void *stream);
+
+/* Sparse decode attention over the kept tokens [R3-2.3 steps 6-7].
+ *   q         [B][H][Dh]  kv_dtype, one decode query per sequence
+ *   K, V      chunk_ids != NULL: the full caches [sum L_b][H][Dh], read through the ids;
+ *             chunk_ids == NULL: resident buffers [sum k_b*C][H][Dh] (lsa_gather_kv output)
+ *   out       [B][H][Dh]  float32: softmax(q.K^T / sqrt(Dh)) V over the kept tokens
+ *   lse       [B][H]      float32 natural-log sum of exp of the scaled logits, or NULL
+ * Split-K flash-decode with fp32 online softmax and a log-sum-exp merge. */
+LSA_API lsa_status lsa_sparse_decode_attn(const lsa_dims *dims, const void *q, const void *K,
+                                  const void *V, const int32_t *chunk_ids, float *out,
+                                  float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/* The fused step: score -> top-k -> attention over the kept chunks, reading K/V
+ * through the kept ids (no resident copy is materialised) [R3-2.3 steps 4-7].
+ * Arguments as above; chunk_ids_out [sum k_b] receives the kept ids; the scores
+ * live in the workspace. Four kernels chained with programmatic dependent launch. */
+LSA_API lsa_status lsa_decode_step(const lsa_dims *dims, const void *q_emb, const void *chunk_emb,
+                           const void *q, const void *K, const void *V,
+                           int32_t *chunk_ids_out, float *out, float *lse,
+                           void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronise `stream`, read the sticky device error word of `ws`, clear it, and
+ * return LSA_OK or the first device error (NONFINITE, BAD_ID, TIMEOUT, in that order). */
+LSA_API lsa_status lsa_get_device_status(void *ws, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H_ */

@@ -1,0 +1,15 @@
+"""Lookahead Sparse Attention (LSA) decode step for B200 (sm_100a).
+
+The chunk-scoring, top-k, gather and sparse flash-decode kernels live in
+``liblsa_b200.so`` (sources in ``csrc/``, C ABI in ``include/lsa.h``);
+``abi`` is the thin ctypes binding with the same entry-point names. The library
+must be built (``learned_sparse_kv_decode_b200.build.build()``): there is no
+fallback when it is missing.
+"""
+from .abi import (  # noqa: F401
+    Dims, LsaError, alloc_workspace, header_symbols, lsa_abi_version, lsa_decode_step,
+    lsa_gather_kv, lsa_get_device_status, lsa_score_chunks, lsa_sparse_decode_attn,
+    lsa_topk_select, lsa_workspace_init, lsa_workspace_size, string,
+    LSA_OK, LSA_ERR_INVALID_ARG, LSA_ERR_WORKSPACE, LSA_ERR_CUDA, LSA_ERR_NONFINITE,
+    LSA_ERR_TIMEOUT, LSA_ERR_UNSUPPORTED, LSA_ERR_BAD_ID, LSA_F32, LSA_BF16,
+)

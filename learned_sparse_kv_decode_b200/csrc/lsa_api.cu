@@ -1,0 +1,282 @@
+// lsa_api.cu - the C ABI (include/lsa.h): host-side validation, launch plans,
+// workspace layout and the kernel launches of the LSA decode step.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "lsa_device.cuh"
+
+namespace lsa {
+cudaError_t launch_score(const lsa_dims& d, const SeqTable& tab, int max_n, const void* q_emb,
+                         const void* chunk_emb, float* scores, uint32_t* err, int num_sms,
+                         cudaStream_t stream, bool pdl);
+bool score_uses_umma(const lsa_dims& d);
+cudaError_t launch_topk(const lsa_dims& d, const SeqTable& tab, int max_n, const float* scores,
+                        int32_t* ids, uint32_t* err, cudaStream_t stream, bool pdl);
+cudaError_t launch_gather(const lsa_dims& d, const SeqTable& tab, const void* K, const void* V,
+                          const int32_t* ids, void* K_res, void* V_res, uint32_t* err,
+                          cudaStream_t stream);
+cudaError_t attn_ctas_per_device(lsa_dtype kv, int num_sms, int* out);
+cudaError_t launch_attention(const lsa_dims& d, const SeqTable& tab, int ctas_per_device,
+                             const void* q, const void* K, const void* V, const int32_t* ids,
+                             float* part_o, float* part_ml, float* out, float* lse, uint32_t* err,
+                             cudaStream_t stream, bool pdl);
+}  // namespace lsa
+
+using namespace lsa;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready;
+    int sms;
+    int attn_ctas[2];  // per kv dtype (LSA_F32, LSA_BF16)
+};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+// SM count and attention CTAs per device, computed once per device.
+lsa_status device_info(DeviceInfo* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LSA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    DeviceInfo& di = g_dev[dev];
+    if (!di.ready) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return LSA_ERR_CUDA;
+        di.sms = sms;
+        if (attn_ctas_per_device(LSA_F32, sms, &di.attn_ctas[LSA_F32]) != cudaSuccess) return LSA_ERR_CUDA;
+        if (attn_ctas_per_device(LSA_BF16, sms, &di.attn_ctas[LSA_BF16]) != cudaSuccess) return LSA_ERR_CUDA;
+        di.ready = true;
+    }
+    *out = di;
+    return LSA_OK;
+}
+
+bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Prepared {
+    SeqTable tab;
+    int max_n;
+    int64_t total_chunks;
+    int64_t total_kept;
+};
+
+// Validate the shape and build the per-sequence table.
+lsa_status prepare(const lsa_dims* d, Prepared* p) {
+    if (d == nullptr || p == nullptr) return LSA_ERR_INVALID_ARG;
+    if (d->B < 1 || d->B > LSA_MAX_BATCH) return LSA_ERR_INVALID_ARG;
+    if (d->Q < 1 || d->Q > 256 || d->E < 1) return LSA_ERR_INVALID_ARG;
+    if (d->emb_dtype != LSA_F32 && d->emb_dtype != LSA_BF16) return LSA_ERR_INVALID_ARG;
+    if (d->kv_dtype != LSA_F32 && d->kv_dtype != LSA_BF16) return LSA_ERR_INVALID_ARG;
+    if (d->Dh != LSA_HEAD_DIM) return LSA_ERR_UNSUPPORTED;
+    if (!is_pow2(d->H) || d->H > 128) return LSA_ERR_UNSUPPORTED;
+    if (!is_pow2(d->chunk_len) || d->chunk_len < 8 || d->chunk_len > 1024) return LSA_ERR_UNSUPPORTED;
+    const int es = d->emb_dtype == LSA_BF16 ? 2 : 4;
+    const int64_t row_bytes = (int64_t)d->E * es;
+    if (row_bytes % 16 != 0) return LSA_ERR_UNSUPPORTED;
+    const int64_t pieces = row_bytes / 16;
+    if (!((pieces <= 32 && is_pow2(pieces)) || pieces % 32 == 0)) return LSA_ERR_UNSUPPORTED;
+    if (!score_uses_umma(*d) && (int64_t)d->Q * d->E * 4 > 200 * 1024) return LSA_ERR_UNSUPPORTED;
+
+    SeqTable& t = p->tab;
+    std::memset(&t, 0, sizeof(t));
+    t.B = d->B;
+    t.C = d->chunk_len;
+    int64_t chunks = 0, kept = 0;
+    int max_n = 0;
+    for (int b = 0; b < d->B; ++b) {
+        int64_t n;
+        if (d->chunk_offsets) {
+            if (b == 0 && d->chunk_offsets[0] != 0) return LSA_ERR_INVALID_ARG;
+            n = d->chunk_offsets[b + 1] - d->chunk_offsets[b];
+        } else {
+            n = d->N;
+        }
+        const int64_t k = d->k_per_seq ? d->k_per_seq[b] : d->k;
+        if (n < 1 || k < 1 || k > n) return LSA_ERR_INVALID_ARG;
+        t.chunk_off[b] = (int32_t)chunks;
+        t.kept_off[b] = (int32_t)kept;
+        chunks += n;
+        kept += k;
+        if (chunks > (1ll << 30) || kept > (1ll << 30)) return LSA_ERR_UNSUPPORTED;
+        if (n > max_n) max_n = (int)n;
+    }
+    t.chunk_off[d->B] = (int32_t)chunks;
+    t.kept_off[d->B] = (int32_t)kept;
+    p->max_n = max_n;
+    p->total_chunks = chunks;
+    p->total_kept = kept;
+    return LSA_OK;
+}
+
+struct WsLayout {
+    size_t scores, part_o, part_ml, total;
+};
+
+WsLayout ws_layout(const lsa_dims* d, const Prepared& p, const DeviceInfo& di) {
+    WsLayout w;
+    const int slots = di.attn_ctas[d->kv_dtype] + d->B;
+    w.scores = kWsHeader;
+    w.part_o = align256(w.scores + (size_t)p.total_chunks * 4);
+    w.part_ml = align256(w.part_o + (size_t)slots * d->H * LSA_HEAD_DIM * 4);
+    w.total = align256(w.part_ml + (size_t)slots * d->H * 2 * 4);
+    return w;
+}
+
+// Validation shared by every call that takes a workspace.
+lsa_status prepare_ws(const lsa_dims* d, void* ws, size_t ws_bytes, Prepared* p, DeviceInfo* di,
+                      WsLayout* w) {
+    lsa_status s = prepare(d, p);
+    if (s != LSA_OK) return s;
+    if (!aligned16(ws)) return LSA_ERR_INVALID_ARG;
+    s = device_info(di);
+    if (s != LSA_OK) return s;
+    *w = ws_layout(d, *p, *di);
+    if (ws_bytes < w->total) return LSA_ERR_WORKSPACE;
+    return LSA_OK;
+}
+
+inline uint8_t* at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
+inline lsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LSA_OK : LSA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int lsa_abi_version(void) { return LSA_ABI_VERSION; }
+
+const char* lsa_status_string(lsa_status s) {
+    switch (s) {
+        case LSA_OK: return "LSA_OK";
+        case LSA_ERR_INVALID_ARG: return "LSA_ERR_INVALID_ARG: invalid argument";
+        case LSA_ERR_WORKSPACE: return "LSA_ERR_WORKSPACE: workspace too small";
+        case LSA_ERR_CUDA: return "LSA_ERR_CUDA: CUDA runtime error";
+        case LSA_ERR_NONFINITE: return "LSA_ERR_NONFINITE: non-finite chunk score";
+        case LSA_ERR_TIMEOUT: return "LSA_ERR_TIMEOUT: a bounded device wait gave up";
+        case LSA_ERR_UNSUPPORTED: return "LSA_ERR_UNSUPPORTED: shape not implemented";
+        case LSA_ERR_BAD_ID: return "LSA_ERR_BAD_ID: kept chunk id out of range";
+    }
+    return "LSA_ERR_?: unknown status";
+}
+
+lsa_status lsa_workspace_size(const lsa_dims* dims, size_t* bytes) {
+    if (bytes == nullptr) return LSA_ERR_INVALID_ARG;
+    Prepared p;
+    lsa_status s = prepare(dims, &p);
+    if (s != LSA_OK) return s;
+    DeviceInfo di;
+    s = device_info(&di);
+    if (s != LSA_OK) return s;
+    *bytes = ws_layout(dims, p, di).total;
+    return LSA_OK;
+}
+
+lsa_status lsa_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+    if (!aligned16(ws) || ws_bytes < kWsHeader) return LSA_ERR_INVALID_ARG;
+    return cuda_status(cudaMemsetAsync(ws, 0, kWsHeader, static_cast<cudaStream_t>(stream)));
+}
+
+lsa_status lsa_score_chunks(const lsa_dims* dims, const void* q_emb, const void* chunk_emb,
+                            float* scores, void* ws, size_t ws_bytes, void* stream) {
+    Prepared p;
+    DeviceInfo di;
+    WsLayout w;
+    lsa_status s = prepare_ws(dims, ws, ws_bytes, &p, &di, &w);
+    if (s != LSA_OK) return s;
+    if (!aligned16(q_emb) || !aligned16(chunk_emb) || !aligned16(scores)) return LSA_ERR_INVALID_ARG;
+    return cuda_status(launch_score(*dims, p.tab, p.max_n, q_emb, chunk_emb, scores,
+                                    reinterpret_cast<uint32_t*>(ws), di.sms,
+                                    static_cast<cudaStream_t>(stream), false));
+}
+
+lsa_status lsa_topk_select(const lsa_dims* dims, const float* scores, int32_t* chunk_ids, void* ws,
+                           size_t ws_bytes, void* stream) {
+    Prepared p;
+    DeviceInfo di;
+    WsLayout w;
+    lsa_status s = prepare_ws(dims, ws, ws_bytes, &p, &di, &w);
+    if (s != LSA_OK) return s;
+    if (!aligned16(scores) || !aligned16(chunk_ids)) return LSA_ERR_INVALID_ARG;
+    return cuda_status(launch_topk(*dims, p.tab, p.max_n, scores, chunk_ids,
+                                   reinterpret_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream),
+                                   false));
+}
+
+lsa_status lsa_gather_kv(const lsa_dims* dims, const void* K, const void* V, const int32_t* chunk_ids,
+                         void* K_res, void* V_res, void* ws, size_t ws_bytes, void* stream) {
+    Prepared p;
+    DeviceInfo di;
+    WsLayout w;
+    lsa_status s = prepare_ws(dims, ws, ws_bytes, &p, &di, &w);
+    if (s != LSA_OK) return s;
+    if (!aligned16(K) || !aligned16(V) || !aligned16(chunk_ids) || !aligned16(K_res) || !aligned16(V_res))
+        return LSA_ERR_INVALID_ARG;
+    return cuda_status(launch_gather(*dims, p.tab, K, V, chunk_ids, K_res, V_res,
+                                     reinterpret_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream)));
+}
+
+lsa_status lsa_sparse_decode_attn(const lsa_dims* dims, const void* q, const void* K, const void* V,
+                                  const int32_t* chunk_ids, float* out, float* lse, void* ws,
+                                  size_t ws_bytes, void* stream) {
+    Prepared p;
+    DeviceInfo di;
+    WsLayout w;
+    lsa_status s = prepare_ws(dims, ws, ws_bytes, &p, &di, &w);
+    if (s != LSA_OK) return s;
+    if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return LSA_ERR_INVALID_ARG;
+    if (chunk_ids != nullptr && !aligned16(chunk_ids)) return LSA_ERR_INVALID_ARG;
+    if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LSA_ERR_INVALID_ARG;
+    return cuda_status(launch_attention(*dims, p.tab, di.attn_ctas[dims->kv_dtype], q, K, V, chunk_ids,
+                                        reinterpret_cast<float*>(at(ws, w.part_o)),
+                                        reinterpret_cast<float*>(at(ws, w.part_ml)), out, lse,
+                                        reinterpret_cast<uint32_t*>(ws),
+                                        static_cast<cudaStream_t>(stream), false));
+}
+
+lsa_status lsa_decode_step(const lsa_dims* dims, const void* q_emb, const void* chunk_emb,
+                           const void* q, const void* K, const void* V, int32_t* chunk_ids_out,
+                           float* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+    Prepared p;
+    DeviceInfo di;
+    WsLayout w;
+    lsa_status s = prepare_ws(dims, ws, ws_bytes, &p, &di, &w);
+    if (s != LSA_OK) return s;
+    if (!aligned16(q_emb) || !aligned16(chunk_emb) || !aligned16(q) || !aligned16(K) ||
+        !aligned16(V) || !aligned16(chunk_ids_out) || !aligned16(out))
+        return LSA_ERR_INVALID_ARG;
+    if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LSA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+    float* scores = reinterpret_cast<float*>(at(ws, w.scores));
+    cudaError_t e = launch_score(*dims, p.tab, p.max_n, q_emb, chunk_emb, scores, err, di.sms, st, false);
+    if (e != cudaSuccess) return LSA_ERR_CUDA;
+    e = launch_topk(*dims, p.tab, p.max_n, scores, chunk_ids_out, err, st, true);
+    if (e != cudaSuccess) return LSA_ERR_CUDA;
+    e = launch_attention(*dims, p.tab, di.attn_ctas[dims->kv_dtype], q, K, V, chunk_ids_out,
+                         reinterpret_cast<float*>(at(ws, w.part_o)),
+                         reinterpret_cast<float*>(at(ws, w.part_ml)), out, lse, err, st, true);
+    return cuda_status(e);
+}
+
+lsa_status lsa_get_device_status(void* ws, void* stream) {
+    if (!aligned16(ws)) return LSA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return LSA_ERR_CUDA;
+    uint32_t word = 0;
+    if (cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return LSA_ERR_CUDA;
+    if (word != 0 && cudaMemset(ws, 0, sizeof(word)) != cudaSuccess) return LSA_ERR_CUDA;
+    if (word & kErrNonFinite) return LSA_ERR_NONFINITE;
+    if (word & kErrBadId) return LSA_ERR_BAD_ID;
+    if (word & kErrTimeout) return LSA_ERR_TIMEOUT;
+    return LSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,340 @@
+// score.cu - chunk relevance scores of the Neural Memory Indexer.
+//
+// FlashMemory-DeepSeek-V4 (review on dimensionstp.github.io, section 3-2 (2);
+// arXiv abstract): the indexer is a dual encoder, so a chunk's relevance is the
+// inner product of the query-side embedding and the chunk-side embedding. With
+// the ~64-token lookahead window (review, section 3-2 (3)) there are Q query
+// embeddings per sequence and a chunk's score is the max over them (the same
+// max the review gives for combining per-layer scores).
+//
+//   scores[i] = max_{j < Q} sum_e q_emb[b][j][e] * chunk_emb[i][e]      (fp32 accumulate)
+//
+// Two kernels:
+//  * k_score_stream - Q small / fp32: an HBM-bound stream over the chunk
+//    embeddings with 128-bit loads, the query held in registers, and a warp
+//    shuffle reduction per row.
+//  * k_score_umma   - Q > 1 with bf16 embeddings: a tcgen05 tensor-core GEMM,
+//    D[128 x Qp] = A[128 chunks x E] * B[Qp queries x E]^T accumulated in TMEM,
+//    followed by a per-row max in the epilogue (tcgen05.ld).
+#include "lsa_device.cuh"
+
+namespace lsa {
+
+// ============================================================== CUDA-core stream
+template <bool BF16>
+__device__ __forceinline__ void unpack16(const uint4& v, float (&x)[8]) {
+    if constexpr (BF16) {
+        x[0] = bf16lo(v.x); x[1] = bf16hi(v.x); x[2] = bf16lo(v.y); x[3] = bf16hi(v.y);
+        x[4] = bf16lo(v.z); x[5] = bf16hi(v.z); x[6] = bf16lo(v.w); x[7] = bf16hi(v.w);
+    } else {
+        x[0] = __uint_as_float(v.x); x[1] = __uint_as_float(v.y);
+        x[2] = __uint_as_float(v.z); x[3] = __uint_as_float(v.w);
+    }
+}
+
+constexpr int kScoreThreads = 256;
+constexpr int kScoreUnroll = 8;
+
+// grid (row blocks, B); dynamic smem: Q*E floats (the queries of sequence b).
+template <bool BF16>
+__global__ void __launch_bounds__(kScoreThreads)
+k_score_stream(const uint8_t* __restrict__ q_emb, const uint8_t* __restrict__ emb,
+               float* __restrict__ scores, const SeqTable tab, int Q, int E, int rows_per_cta) {
+    extern __shared__ float sq[];
+    constexpr int ES = BF16 ? 2 : 4;
+    constexpr int VEC = 16 / ES;  // elements per 16-byte piece
+    const int b = blockIdx.y;
+    const int n_b = tab.chunk_off[b + 1] - tab.chunk_off[b];
+    const int r0 = blockIdx.x * rows_per_cta;
+    pdl_trigger();
+    if (r0 >= n_b) return;
+    const int r1 = min(n_b, r0 + rows_per_cta);
+
+    const size_t qbase = (size_t)b * Q * E;
+    for (int i = threadIdx.x; i < Q * E; i += blockDim.x) {
+        if constexpr (BF16) {
+            const uint16_t h = reinterpret_cast<const uint16_t*>(q_emb)[qbase + i];
+            sq[i] = __uint_as_float((uint32_t)h << 16);
+        } else {
+            sq[i] = reinterpret_cast<const float*>(q_emb)[qbase + i];
+        }
+    }
+    __syncthreads();
+
+    const int P = E / VEC;            // 16-byte pieces per row
+    const int LPR = P < 32 ? P : 32;  // lanes per row
+    const int RPW = 32 / LPR;         // rows per warp step
+    const int PPL = P / LPR;          // pieces per lane
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sub = lane / LPR, li = lane % LPR;
+    const int nwarps = blockDim.x >> 5;
+    const size_t row_bytes = (size_t)E * ES;
+    const uint8_t* base = emb + (size_t)tab.chunk_off[b] * row_bytes;
+    float* out = scores + tab.chunk_off[b];
+    const int step = nwarps * RPW;
+
+    // The loop bound is warp-uniform (every lane joins the shuffles); rows past r1 are masked.
+    for (int wrow = r0 + warp * RPW; wrow < r1; wrow += step * kScoreUnroll) {
+        const int row0 = wrow + sub;
+        float best[kScoreUnroll];
+#pragma unroll
+        for (int u = 0; u < kScoreUnroll; ++u) best[u] = -INFINITY;
+        for (int j = 0; j < Q; ++j) {
+            float acc[kScoreUnroll];
+#pragma unroll
+            for (int u = 0; u < kScoreUnroll; ++u) acc[u] = 0.f;
+            for (int p = 0; p < PPL; ++p) {
+                const int piece = li + p * LPR;
+                uint4 v[kScoreUnroll];
+#pragma unroll
+                for (int u = 0; u < kScoreUnroll; ++u) {
+                    const int row = row0 + u * step;
+                    v[u] = row < r1 ? ld_stream16(base + (size_t)row * row_bytes + (size_t)piece * 16)
+                                    : make_uint4(0, 0, 0, 0);
+                }
+                const float* qp = sq + j * E + piece * VEC;
+                float qv[8];
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) qv[e] = qp[e];
+#pragma unroll
+                for (int u = 0; u < kScoreUnroll; ++u) {
+                    float x[8];
+                    unpack16<BF16>(v[u], x);
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) acc[u] = fmaf(qv[e], x[e], acc[u]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kScoreUnroll; ++u) {
+                for (int off = LPR >> 1; off > 0; off >>= 1)
+                    acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], off);
+                best[u] = fmaxf(best[u], acc[u]);
+            }
+        }
+        if (li == 0) {
+#pragma unroll
+            for (int u = 0; u < kScoreUnroll; ++u) {
+                const int row = row0 + u * step;
+                if (row < r1) out[row] = best[u];
+            }
+        }
+    }
+}
+
+// ============================================================== tcgen05 GEMM + row max
+// Shared-memory operand layout: K-major, no swizzle ("interleaved" canonical
+// layout). An 8-row x 16-byte core matrix is 128 contiguous bytes; core
+// matrices adjacent along K are LBO = 128 bytes apart, and 8-row groups are
+// SBO = E*16 bytes apart. Piece p = ((g*KC + c)*8 + r) sits at byte p*16, so a
+// warp's 16-byte stores are contiguous.
+__device__ __forceinline__ uint64_t umma_desc_k_noswizzle(uint32_t saddr, uint32_t lbo,
+                                                          uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+    // base offset 0, absolute LBO mode off, layout type 0 = no swizzle
+    return d;
+}
+
+// Instruction descriptor of kind::f16: bf16 A and B, fp32 D, both K-major, M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N) {
+    return (1u << 4)                         // D format: f32
+           | (1u << 7)                       // A format: bf16
+           | (1u << 10)                      // B format: bf16
+           | ((uint32_t)(N >> 3) << 17)      // N / 8
+           | ((uint32_t)(M >> 4) << 24);     // M / 16
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+constexpr int kUmmaM = 128;
+
+// grid (ceil(maxN/128), B), 128 threads; dynamic smem: A (128*E*2) + B (Np*E*2), 1 KiB aligned.
+__global__ void __launch_bounds__(128)
+k_score_umma(const uint16_t* __restrict__ q_emb, const uint16_t* __restrict__ emb,
+             float* __restrict__ scores, const SeqTable tab, int Q, int Np, int E,
+             uint32_t tmem_cols, uint32_t* err) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    __shared__ __align__(8) uint64_t mma_bar;
+    __shared__ uint32_t tmem_slot;
+
+    const int b = blockIdx.y;
+    const int n_b = tab.chunk_off[b + 1] - tab.chunk_off[b];
+    const int r0 = blockIdx.x * kUmmaM;
+    pdl_trigger();
+    if (r0 >= n_b) return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + (size_t)kUmmaM * E * 2;
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&tmem_slot)),
+                     "r"(tmem_cols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        mbar_init(smem_u32(&mma_bar), 1);
+        fence_mbar_init();
+    }
+
+    // ---- stage A (128 chunk rows) and B (Np query rows, zero-padded) into the core-matrix layout
+    const int KC = E / 8;  // 16-byte pieces per row
+    const uint16_t* gA = emb + ((size_t)tab.chunk_off[b] + r0) * E;
+    const int rows_a = min(kUmmaM, n_b - r0);
+    const int pieces_a = kUmmaM * KC;
+    for (int p0 = tid; p0 < pieces_a; p0 += 128 * 4) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int p = p0 + u * 128;
+            v[u] = make_uint4(0, 0, 0, 0);
+            if (p < pieces_a) {
+                const int r = p & 7, c = (p >> 3) % KC, g = (p >> 3) / KC;
+                const int row = g * 8 + r;
+                if (row < rows_a) v[u] = ld_stream16(gA + (size_t)row * E + c * 8);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int p = p0 + u * 128;
+            if (p < pieces_a) *reinterpret_cast<uint4*>(sA + (size_t)p * 16) = v[u];
+        }
+    }
+    const uint16_t* gB = q_emb + (size_t)b * Q * E;
+    const int pieces_b = Np * KC;
+    for (int p = tid; p < pieces_b; p += 128) {
+        const int r = p & 7, c = (p >> 3) % KC, g = (p >> 3) / KC;
+        const int row = g * 8 + r;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (row < Q) v = *reinterpret_cast<const uint4*>(gB + (size_t)row * E + c * 8);
+        *reinterpret_cast<uint4*>(sB + (size_t)p * 16) = v;
+    }
+    // generic-proxy smem writes -> visible to the tensor core (async proxy)
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_d = tmem_slot;
+
+    if (tid == 0) {
+        const uint32_t idesc = umma_idesc_bf16_f32(kUmmaM, Np);
+        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+        const uint32_t sbo = (uint32_t)E * 16;
+        for (int ks = 0; ks < E / 16; ++ks) {
+            const uint64_t ad = umma_desc_k_noswizzle(a0 + ks * 256, 128, sbo);
+            const uint64_t bd = umma_desc_k_noswizzle(b0 + ks * 256, 128, sbo);
+            const uint32_t accum = ks > 0 ? 1u : 0u;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "setp.ne.b32 p, %4, 0;\n\t"
+                "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+                "l"(ad), "l"(bd), "r"(idesc), "r"(accum)
+                : "memory");
+        }
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32(&mma_bar))
+                     : "memory");
+    }
+    // warp-uniform: the tcgen05.ld below is .sync.aligned
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&mma_bar), 0, err));
+    tc_fence_after();
+
+    // ---- epilogue: row r0 + 32*warp + lane lives in TMEM lane 32*warp + lane
+    float best = -INFINITY;
+    if (ok) {
+        const uint32_t taddr = tmem_d + ((uint32_t)(warp * 32) << 16);
+        for (int c0 = 0; c0 < Np; c0 += 16) {
+            uint32_t r[16];
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                  "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+                  "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                : "r"(taddr + (uint32_t)c0));
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (c0 + i < Q) best = fmaxf(best, __uint_as_float(r[i]));
+        }
+        const int row = r0 + warp * 32 + lane;
+        if (row < n_b) scores[tab.chunk_off[b] + row] = best;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d),
+                     "r"(tmem_cols)
+                     : "memory");
+    }
+}
+
+// ============================================================== launchers
+// A and B tiles plus 4 KiB of slack after them (never read when the descriptors are right).
+size_t score_umma_smem(int E, int Np) { return (size_t)(kUmmaM + Np) * E * 2 + 4096; }
+
+bool score_uses_umma(const lsa_dims& d) {
+    return d.Q > 1 && d.emb_dtype == LSA_BF16 && d.E % 16 == 0 && d.E <= 256 && d.Q <= 256;
+}
+
+cudaError_t launch_score(const lsa_dims& d, const SeqTable& tab, int max_n, const void* q_emb,
+                         const void* chunk_emb, float* scores, uint32_t* err, int num_sms,
+                         cudaStream_t stream, bool pdl) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+
+    if (score_uses_umma(d)) {
+        const int Np = (d.Q + 15) / 16 * 16;
+        uint32_t cols = 32;
+        while ((int)cols < Np) cols <<= 1;
+        const size_t smem = score_umma_smem(d.E, Np);
+        cudaError_t e = cudaFuncSetAttribute(k_score_umma, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        cfg.gridDim = dim3((max_n + kUmmaM - 1) / kUmmaM, d.B, 1);
+        cfg.blockDim = dim3(128, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        return cudaLaunchKernelEx(&cfg, k_score_umma, (const uint16_t*)q_emb,
+                                  (const uint16_t*)chunk_emb, scores, tab, d.Q, Np, d.E, cols, err);
+    }
+    const int es = d.emb_dtype == LSA_BF16 ? 2 : 4;
+    const int P = d.E * es / 16;
+    const int LPR = P < 32 ? P : 32;
+    const int rows_step = (kScoreThreads / 32) * (32 / LPR) * kScoreUnroll;
+    int total_rows = tab.chunk_off[d.B];
+    int want = (total_rows + 4 * num_sms - 1) / (4 * num_sms);
+    int rpc = (want + rows_step - 1) / rows_step * rows_step;
+    if (rpc < rows_step) rpc = rows_step;
+    cfg.gridDim = dim3((max_n + rpc - 1) / rpc, d.B, 1);
+    cfg.blockDim = dim3(kScoreThreads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)d.Q * d.E * sizeof(float);
+    if (d.emb_dtype == LSA_BF16) {
+        cudaError_t e = cudaFuncSetAttribute(k_score_stream<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)cfg.dynamicSmemBytes);
+        if (e != cudaSuccess) return e;
+        return cudaLaunchKernelEx(&cfg, k_score_stream<true>, (const uint8_t*)q_emb,
+                                  (const uint8_t*)chunk_emb, scores, tab, d.Q, d.E, rpc);
+    }
+    cudaError_t e = cudaFuncSetAttribute(k_score_stream<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)cfg.dynamicSmemBytes);
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&cfg, k_score_stream<false>, (const uint8_t*)q_emb,
+                              (const uint8_t*)chunk_emb, scores, tab, d.Q, d.E, rpc);
+}
+
+}  // namespace lsa

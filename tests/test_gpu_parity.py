@@ -1,0 +1,323 @@
+"""GPU parity: every C-ABI call against the float64 oracle on the same seeded inputs.
+
+Small cases are compared element by element (several tiles and ragged tails);
+the full-size decode workloads are run in the same launch configuration the
+benchmark times and compared on all chunk ids and on sampled (sequence, head)
+outputs, which the oracle recomputes from regenerated K/V rows."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import datagen
+import oracle
+from datagen import device as dgdev
+from tests import _gpu as G
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lsa():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from learned_sparse_kv_decode_b200 import build
+    build.build()
+    import learned_sparse_kv_decode_b200 as m
+    return m
+
+
+def _free():
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------------ input generator
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_device_generator_matches_host(dt):
+    n, first = 100_003, 12_345_678_901
+    t = torch.empty(n, dtype=G.tdtype(dt), device="cuda")
+    dgdev.fill_normal(t, 7, 4, first)
+    host = datagen.normal_f32(7, 4, np.arange(first, first + n, dtype=np.uint64))
+    if dt == "bf16":
+        got = t.view(torch.int16).cpu().numpy().view(np.uint16)
+        np.testing.assert_array_equal(got, datagen.bf16_bits(host))
+    else:
+        np.testing.assert_array_equal(t.cpu().numpy(), host)
+
+
+# ------------------------------------------------------------------ scores
+SCORE_CASES = [
+    dict(name="f32-E64", emb_dtype="f32", E=64, Q=1, N=(40, 72, 1)),
+    dict(name="f32-E128", emb_dtype="f32", E=128, Q=1, N=(300, 1, 77)),
+    dict(name="f32-E256", emb_dtype="f32", E=256, Q=1, N=(129, 64)),
+    dict(name="bf16-E128", emb_dtype="bf16", E=128, Q=1, N=(2048, 5, 333)),
+    dict(name="bf16-E256", emb_dtype="bf16", E=256, Q=1, N=(1000, 17)),
+    dict(name="bf16-E1024", emb_dtype="bf16", E=1024, Q=1, N=(70, 3)),
+    dict(name="f32-Q3", emb_dtype="f32", E=128, Q=3, N=(90, 31)),
+    dict(name="umma-Q64-E256", emb_dtype="bf16", E=256, Q=64, N=(300, 129, 128, 1)),
+    dict(name="umma-Q64-E128", emb_dtype="bf16", E=128, Q=64, N=(513, 7)),
+    dict(name="umma-Q3-E64", emb_dtype="bf16", E=64, Q=3, N=(260,)),
+    dict(name="umma-Q200-E128", emb_dtype="bf16", E=128, Q=200, N=(140, 120)),
+]
+
+
+@pytest.mark.parametrize("case", SCORE_CASES, ids=lambda c: c["name"])
+def test_score_chunks_parity(lsa, case):
+    N = case["N"]
+    w = datagen.small_workload(B=len(N), N=N, E=case["E"], Q=case["Q"], k=[1] * len(N), H=4,
+                               emb_dtype=case["emb_dtype"], seed=21, plant="copy_query" if case["Q"] > 1 else "copy")
+    dw = G.DeviceWorkload(w, lsa, with_kv=False)
+    lsa.lsa_score_chunks(dw.dims, dw.q_emb, dw.chunk_emb, dw.scores, dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_OK
+    got = dw.scores.cpu().numpy()
+    off = w.chunk_offsets
+    for b in range(w.B):
+        qf, ef = dw.q_emb_f(b), dw.emb_f(b)
+        ref = oracle.chunk_scores(qf, ef)
+        G.check_scores(got[off[b]:off[b + 1]], ref, G.score_tolerance(qf, ef))
+
+
+# ------------------------------------------------------------------ top-k
+def _tie_scores(n, seed, levels=4.0):
+    x = datagen.normal_f32(seed, 1, np.arange(n))
+    return (np.round(x * levels) / levels).astype(np.float32)  # many exact ties
+
+
+@pytest.mark.parametrize("N,k", [((1,), (1,)), ((7, 64), (3, 64)), ((1000, 999), (1, 998)),
+                                 ((5000, 16384), (700, 2212)), ((60000,), (6000,))])
+def test_topk_bit_exact_with_ties(lsa, N, k):
+    w = datagen.small_workload(B=len(N), N=N, k=k, E=64)
+    dims = G.dims_of(w, lsa)
+    ws = lsa.alloc_workspace(dims)
+    s = np.concatenate([_tie_scores(n, 100 + i) for i, n in enumerate(N)])
+    s[::17] = -s[::17]
+    ids = torch.empty(w.total_kept, dtype=torch.int32, device="cuda")
+    lsa.lsa_topk_select(dims, torch.from_numpy(s).cuda(), ids, ws)
+    assert lsa.lsa_get_device_status(ws) == lsa.LSA_OK
+    got = ids.cpu().numpy()
+    off, koff = w.chunk_offsets, w.k_offsets
+    for b in range(w.B):
+        ref = oracle.topk(s[off[b]:off[b + 1]].astype(np.float64), k[b])
+        np.testing.assert_array_equal(got[koff[b]:koff[b + 1]], ref)
+
+
+def test_topk_signed_zero_and_all_equal(lsa):
+    w = datagen.small_workload(B=3, N=(8, 10, 6), k=(7, 4, 6), E=64)
+    dims = G.dims_of(w, lsa)
+    ws = lsa.alloc_workspace(dims)
+    s = np.array([3, 7, 7, 1, 7, -0.0, 0.0, 5] + [2.5] * 10 + [-1, -2, -3, -0.0, -5, -6], np.float32)
+    ids = torch.empty(w.total_kept, dtype=torch.int32, device="cuda")
+    lsa.lsa_topk_select(dims, torch.from_numpy(s).cuda(), ids, ws)
+    got = ids.cpu().numpy()
+    np.testing.assert_array_equal(got[:7], [0, 1, 2, 3, 4, 5, 7])
+    np.testing.assert_array_equal(got[7:11], [0, 1, 2, 3])
+    np.testing.assert_array_equal(got[11:], [0, 1, 2, 3, 4, 5])
+
+
+def test_topk_nonfinite_reported(lsa):
+    w = datagen.small_workload(B=1, N=(50,), k=(10,), E=64)
+    dims = G.dims_of(w, lsa)
+    ws = lsa.alloc_workspace(dims)
+    s = _tie_scores(50, 3)
+    s[11] = np.nan
+    ids = torch.empty(10, dtype=torch.int32, device="cuda")
+    lsa.lsa_topk_select(dims, torch.from_numpy(s).cuda(), ids, ws)
+    assert lsa.lsa_get_device_status(ws) == lsa.LSA_ERR_NONFINITE
+    got = ids.cpu().numpy()
+    assert got.min() >= 0 and got.max() < 50 and 11 not in got
+    assert lsa.lsa_get_device_status(ws) == lsa.LSA_OK  # the word was cleared
+
+
+# ------------------------------------------------------------------ gather
+@pytest.mark.parametrize("kv_dtype,H,C", [("f32", 8, 64), ("bf16", 16, 64), ("bf16", 2, 32), ("f32", 1, 8)])
+def test_gather_bit_exact(lsa, kv_dtype, H, C):
+    w = datagen.small_workload(B=3, N=(9, 4, 13), k=(3, 4, 5), E=64, H=H, C=C, kv_dtype=kv_dtype)
+    dw = G.DeviceWorkload(w, lsa)
+    rng = np.random.default_rng(5)
+    ids = np.concatenate([np.sort(rng.permutation(n)[:k]) for n, k in zip(w.N, w.k)]).astype(np.int32)
+    Kr = torch.empty((w.total_kept * C, H, w.Dh), dtype=G.tdtype(kv_dtype), device="cuda")
+    Vr = torch.empty_like(Kr)
+    lsa.lsa_gather_kv(dw.dims, dw.K, dw.V, torch.from_numpy(ids).cuda(), Kr, Vr, dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_OK
+    koff = w.k_offsets
+    Kg, Vg = Kr.float().cpu().numpy(), Vr.float().cpu().numpy()
+    for b in range(w.B):
+        tok = oracle.kept_tokens(ids[koff[b]:koff[b + 1]], C)
+        rows = slice(koff[b] * C, koff[b + 1] * C)
+        np.testing.assert_array_equal(Kg[rows], dw.kv_f("K", b, tok))
+        np.testing.assert_array_equal(Vg[rows], dw.kv_f("V", b, tok))
+
+
+def test_gather_bad_id_reported(lsa):
+    w = datagen.small_workload(B=1, N=(5,), k=(2,), E=64, H=2)
+    dw = G.DeviceWorkload(w, lsa)
+    Kr = torch.zeros((2 * w.C, 2, w.Dh), dtype=torch.float32, device="cuda")
+    Vr = torch.zeros_like(Kr)
+    lsa.lsa_gather_kv(dw.dims, dw.K, dw.V, torch.tensor([1, 5], dtype=torch.int32, device="cuda"), Kr, Vr, dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_ERR_BAD_ID
+    np.testing.assert_array_equal(Kr[:w.C].cpu().numpy(), dw.kv_f("K", 0, np.arange(w.C, 2 * w.C)))
+    assert float(Kr[w.C:].abs().max()) == 0.0
+
+
+# ------------------------------------------------------------------ sparse attention
+ATTN_CASES = [
+    dict(kv_dtype="f32", H=8, C=64, N=(20, 9), k=(6, 9)),
+    dict(kv_dtype="bf16", H=16, C=64, N=(30, 3, 11), k=(10, 1, 11)),
+    dict(kv_dtype="bf16", H=8, C=64, N=(12, 40), k=(12, 5)),
+    dict(kv_dtype="bf16", H=32, C=64, N=(6,), k=(4,)),
+    dict(kv_dtype="bf16", H=1, C=16, N=(50, 2), k=(33, 2)),
+    dict(kv_dtype="f32", H=2, C=8, N=(64,), k=(17,)),
+    dict(kv_dtype="f32", H=16, C=32, N=(10, 10), k=(3, 7)),
+    dict(kv_dtype="bf16", H=4, C=128, N=(7, 5, 9, 1), k=(2, 5, 9, 1)),
+]
+
+
+@pytest.mark.parametrize("mode", ["indexed", "resident"])
+@pytest.mark.parametrize("case", ATTN_CASES, ids=lambda c: f"{c['kv_dtype']}-H{c['H']}-C{c['C']}-B{len(c['N'])}")
+def test_sparse_attention_parity(lsa, case, mode):
+    w = datagen.small_workload(B=len(case["N"]), N=case["N"], k=case["k"], E=64, H=case["H"], C=case["C"],
+                               kv_dtype=case["kv_dtype"], seed=33)
+    dw = G.DeviceWorkload(w, lsa)
+    rng = np.random.default_rng(7)
+    ids = np.concatenate([np.sort(rng.permutation(n)[:k]) for n, k in zip(w.N, w.k)]).astype(np.int32)
+    ids_d = torch.from_numpy(ids).cuda()
+    if mode == "indexed":
+        lsa.lsa_sparse_decode_attn(dw.dims, dw.q, dw.K, dw.V, ids_d, dw.out, dw.lse, dw.ws)
+    else:
+        Kr = torch.empty((w.total_kept * w.C, w.H, w.Dh), dtype=G.tdtype(w.kv_dtype), device="cuda")
+        Vr = torch.empty_like(Kr)
+        lsa.lsa_gather_kv(dw.dims, dw.K, dw.V, ids_d, Kr, Vr, dw.ws)
+        lsa.lsa_sparse_decode_attn(dw.dims, dw.q, Kr, Vr, None, dw.out, dw.lse, dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_OK
+    out, lse = dw.out.cpu().numpy(), dw.lse.cpu().numpy()
+    koff = w.k_offsets
+    for b in range(w.B):
+        ref_o, ref_l = G.oracle_attention(dw, b, ids[koff[b]:koff[b + 1]])
+        np.testing.assert_allclose(out[b], ref_o, rtol=0, atol=G.ATTN_ATOL[w.kv_dtype])
+        np.testing.assert_allclose(out[b], ref_o, rtol=0, atol=1e-4)   # fp32 arithmetic on exact inputs
+        np.testing.assert_allclose(lse[b], ref_l, rtol=0, atol=1e-4)
+
+
+def test_attention_bad_id_reported(lsa):
+    w = datagen.small_workload(B=2, N=(4, 4), k=(2, 2), E=64, H=8)
+    dw = G.DeviceWorkload(w, lsa)
+    ids = torch.tensor([0, 1, 2, -3], dtype=torch.int32, device="cuda")
+    lsa.lsa_sparse_decode_attn(dw.dims, dw.q, dw.K, dw.V, ids, dw.out, None, dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_ERR_BAD_ID
+    ref_o, _ = G.oracle_attention(dw, 0, np.array([0, 1]))
+    np.testing.assert_allclose(dw.out[0].cpu().numpy(), ref_o, rtol=0, atol=1e-4)
+
+
+# ------------------------------------------------------------------ fused decode step
+def _run_step(lsa, dw):
+    lsa.lsa_decode_step(dw.dims, dw.q_emb, dw.chunk_emb, dw.q, dw.K, dw.V, dw.ids, dw.out, dw.lse, dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_OK
+
+
+def _check_step(dw, seqs=None, heads_per_seq=None):
+    w = dw.w
+    got_ids, out, lse = dw.ids.cpu().numpy(), dw.out.cpu().numpy(), dw.lse.cpu().numpy()
+    koff = w.k_offsets
+    seqs = range(w.B) if seqs is None else seqs
+    exempt = 0
+    for b in range(w.B):
+        ref_s = oracle.chunk_scores(dw.q_emb_f(b), dw.emb_f(b))
+        ref_ids = oracle.topk(ref_s, w.k[b])
+        gids = got_ids[koff[b]:koff[b + 1]]
+        exempt += G.check_ids(gids, ref_ids, ref_s, w.k[b])
+        if b not in seqs:
+            continue
+        heads = None if heads_per_seq is None else heads_per_seq(b)
+        ref_o, ref_l = G.oracle_attention(dw, b, gids, heads)
+        got_o = out[b] if heads is None else out[b][heads]
+        got_l = lse[b] if heads is None else lse[b][heads]
+        np.testing.assert_allclose(got_o, ref_o, rtol=0, atol=G.ATTN_ATOL[w.kv_dtype])
+        np.testing.assert_allclose(got_o, ref_o, rtol=0, atol=1e-4)
+        np.testing.assert_allclose(got_l, ref_l, rtol=0, atol=1e-4)
+    return exempt
+
+
+def test_decode_step_tiny_full(lsa):
+    dw = G.DeviceWorkload(datagen.workload("tiny"), lsa)
+    _run_step(lsa, dw)
+    assert _check_step(dw) == 0
+    planted = datagen.planted_positions(dw.w, 0)
+    assert set(planted.tolist()) <= set(dw.ids.cpu().numpy().tolist())
+
+
+STEP_CASES = [
+    dict(B=3, N=(40, 72, 5), k=(5, 9, 5), E=64, H=4, emb_dtype="f32", kv_dtype="f32"),
+    dict(B=2, N=(300, 129), k=(40, 1), E=128, H=16, emb_dtype="bf16", kv_dtype="bf16"),
+    dict(B=4, N=(33, 65, 1, 200), k=(33, 8, 1, 27), E=256, H=8, emb_dtype="bf16", kv_dtype="bf16"),
+    dict(B=1, N=(600,), k=(81,), E=256, Q=64, H=16, emb_dtype="bf16", kv_dtype="bf16", plant="copy_query"),
+    dict(B=2, N=(130, 257), k=(18, 35), E=128, Q=64, H=16, emb_dtype="bf16", kv_dtype="bf16", plant="copy_query"),
+]
+
+
+@pytest.mark.parametrize("case", STEP_CASES, ids=lambda c: f"B{c['B']}-E{c['E']}-Q{c.get('Q', 1)}-H{c['H']}-{c['kv_dtype']}")
+def test_decode_step_small(lsa, case):
+    case = dict(case)
+    w = datagen.small_workload(seed=44, **case)
+    dw = G.DeviceWorkload(w, lsa)
+    _run_step(lsa, dw)
+    _check_step(dw)
+
+
+def test_decode_step_deterministic(lsa):
+    w = datagen.small_workload(B=2, N=(300, 129), k=(40, 7), E=128, H=16, emb_dtype="bf16", kv_dtype="bf16")
+    dw = G.DeviceWorkload(w, lsa)
+    _run_step(lsa, dw)
+    a = (dw.ids.clone(), dw.out.clone(), dw.lse.clone())
+    for _ in range(3):
+        _run_step(lsa, dw)
+        assert torch.equal(a[0], dw.ids) and torch.equal(a[1], dw.out) and torch.equal(a[2], dw.lse)
+
+
+def test_decode_step_keep_all_is_dense_attention(lsa):
+    # k = N: the LSA step is plain dense decode attention (checked against torch SDPA in float64)
+    w = datagen.small_workload(B=2, N=(12, 7), k=(12, 7), E=64, H=8, kv_dtype="f32")
+    dw = G.DeviceWorkload(w, lsa)
+    _run_step(lsa, dw)
+    for b in range(w.B):
+        L = w.L[b]
+        K = torch.from_numpy(dw.kv_f("K", b, np.arange(L)).astype(np.float64)).permute(1, 0, 2)
+        V = torch.from_numpy(dw.kv_f("V", b, np.arange(L)).astype(np.float64)).permute(1, 0, 2)
+        q = torch.from_numpy(dw.q_f(b).astype(np.float64))[:, None, :]
+        ref = torch.nn.functional.scaled_dot_product_attention(q, K, V)[:, 0, :].numpy()
+        np.testing.assert_allclose(dw.out[b].cpu().numpy(), ref, rtol=0, atol=1e-4)
+
+
+# ------------------------------------------------------------------ full-size workloads
+@pytest.mark.parametrize("name", ["128k", "500k", "1m", "mixed"])
+def test_decode_step_full_size(lsa, name):
+    w = datagen.workload(name)
+    dw = G.DeviceWorkload(w, lsa)
+    _run_step(lsa, dw)
+    rng = np.random.default_rng(1)
+    seqs = sorted(set(rng.integers(0, w.B, size=2).tolist()))
+    heads = {b: np.sort(rng.permutation(w.H)[:2]) for b in seqs}
+    _check_step(dw, seqs=seqs, heads_per_seq=lambda b: heads[b])
+    if w.plant == "copy":
+        got = dw.ids.cpu().numpy()
+        for b in range(w.B):
+            kept = set(got[w.k_offsets[b]:w.k_offsets[b + 1]].tolist())
+            assert set(datagen.planted_positions(w, b).tolist()) <= kept
+    del dw
+    _free()
+
+
+# ------------------------------------------------------------------ argument errors
+def test_argument_errors(lsa):
+    w = datagen.small_workload(B=1, N=(8,), k=(2,), E=64, H=4)
+    dw = G.DeviceWorkload(w, lsa)
+    with pytest.raises(lsa.LsaError) as e:
+        lsa.lsa_decode_step(dw.dims, dw.q_emb, dw.chunk_emb, dw.q, dw.K, dw.V, dw.ids, dw.out, dw.lse, dw.ws[:64])
+    assert e.value.status == lsa.LSA_ERR_WORKSPACE
+    raw = torch.empty(dw.scores.numel() + 4, dtype=torch.float32, device="cuda")
+    with pytest.raises(lsa.LsaError) as e:
+        lsa.lsa_score_chunks(dw.dims, dw.q_emb, dw.chunk_emb, raw[1:], dw.ws)  # 4-byte offset: misaligned
+    assert e.value.status == lsa.LSA_ERR_INVALID_ARG
+    with pytest.raises(lsa.LsaError) as e:
+        lsa.lsa_sparse_decode_attn(dw.dims, None, dw.K, dw.V, dw.ids, dw.out, None, dw.ws)
+    assert e.value.status == lsa.LSA_ERR_INVALID_ARG
