@@ -214,6 +214,9 @@ def workload(name: str) -> Workload:
     if name == "128k":
         return Workload("128k", 8, [2048] * 8, 128, 1, [256] * 8, 16, seed=1, plant="copy",
                         plant_count=[32] * 8)
+    if name == "128k-b2":  # the 128K shape with batch 2: a profiling case (2.1 GB of K/V, kept set > L2)
+        return Workload("128k-b2", 2, [2048] * 2, 128, 1, [256] * 2, 16, seed=1, plant="copy",
+                        plant_count=[32] * 2)
     if name == "500k":
         return Workload("500k", 4, [8192] * 4, 256, 1, [819] * 4, 16, seed=2, plant="zipf")
     if name == "1m":
@@ -315,3 +318,18 @@ def kv_rows(w: Workload, which: str, tokens, heads=None) -> np.ndarray:
 def as_f32(a: np.ndarray, dtype: str) -> np.ndarray:
     """Storage array -> exact float32 values (public helper)."""
     return _value(a, dtype)
+
+
+def make_query_variant(w: Workload, r: int) -> dict:
+    """Query embeddings and decode queries of rotation r (r = 0 is make_inputs' own).
+
+    Variant r > 0 draws q_emb and q from seed ``w.seed + 1000 * r``; the chunk
+    embeddings and caches stay those of the workload, so each variant keeps a
+    different set of chunks with the same byte count."""
+    if r == 0:
+        x = make_inputs(w)
+        return {"q_emb": x["q_emb"], "q": x["q"]}
+    seed = w.seed + 1000 * r
+    q_emb = normal_f32(seed, TENSOR_IDS["q_emb"], np.arange(w.B * w.Q * w.E)).reshape(w.B, w.Q, w.E)
+    q = normal_f32(seed, TENSOR_IDS["q"], np.arange(w.B * w.H * w.Dh)).reshape(w.B, w.H, w.Dh)
+    return {"q_emb": _store(q_emb, w.emb_dtype), "q": _store(q, w.kv_dtype)}

@@ -395,13 +395,9 @@ cudaError_t launch_attention(const lsa_dims& d, const SeqTable& tab, int ctas_pe
     cfg.dynamicSmemBytes = L.smem;
     cudaError_t e;
     if (d.kv_dtype == LSA_BF16) {
-        e = cudaFuncSetAttribute(k_attn_split<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem);
-        if (e != cudaSuccess) return e;
         e = cudaLaunchKernelEx(&cfg, k_attn_split<true>, (const uint8_t*)q, (const uint8_t*)K,
                                (const uint8_t*)V, ids, part_o, part_ml, tab, L.ap, err);
     } else {
-        e = cudaFuncSetAttribute(k_attn_split<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem);
-        if (e != cudaSuccess) return e;
         e = cudaLaunchKernelEx(&cfg, k_attn_split<false>, (const uint8_t*)q, (const uint8_t*)K,
                                (const uint8_t*)V, ids, part_o, part_ml, tab, L.ap, err);
     }

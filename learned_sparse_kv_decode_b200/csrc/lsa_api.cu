@@ -19,6 +19,8 @@ cudaError_t launch_gather(const lsa_dims& d, const SeqTable& tab, const void* K,
                           const int32_t* ids, void* K_res, void* V_res, uint32_t* err,
                           cudaStream_t stream);
 cudaError_t attn_ctas_per_device(lsa_dtype kv, int num_sms, int* out);
+cudaError_t score_init_attrs();
+cudaError_t topk_init_attrs();
 cudaError_t launch_attention(const lsa_dims& d, const SeqTable& tab, int ctas_per_device,
                              const void* q, const void* K, const void* V, const int32_t* ids,
                              float* part_o, float* part_ml, float* out, float* lse, uint32_t* err,
@@ -50,6 +52,8 @@ lsa_status device_info(DeviceInfo* out) {
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return LSA_ERR_CUDA;
         di.sms = sms;
+        // kernel attributes are per device: set them here, never inside a launch (graph capture)
+        if (score_init_attrs() != cudaSuccess || topk_init_attrs() != cudaSuccess) return LSA_ERR_CUDA;
         if (attn_ctas_per_device(LSA_F32, sms, &di.attn_ctas[LSA_F32]) != cudaSuccess) return LSA_ERR_CUDA;
         if (attn_ctas_per_device(LSA_BF16, sms, &di.attn_ctas[LSA_BF16]) != cudaSuccess) return LSA_ERR_CUDA;
         di.ready = true;

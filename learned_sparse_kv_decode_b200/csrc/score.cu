@@ -280,6 +280,23 @@ k_score_umma(const uint16_t* __restrict__ q_emb, const uint16_t* __restrict__ em
 }
 
 // ============================================================== launchers
+// Raise the dynamic shared-memory limit of the score kernels (once per device).
+// The limits are the largest requests the launchers make (E <= 256 and Q <= 256 for the
+// tensor-core kernel; Q*E*4 <= 200 KiB for the stream kernel, checked on the host).
+constexpr int kScoreStreamSmemMax = 200 * 1024;
+size_t score_umma_smem(int E, int Np);
+cudaError_t score_init_attrs() {
+    cudaError_t e = cudaFuncSetAttribute(k_score_umma, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)score_umma_smem(256, 256));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_score_stream<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kScoreStreamSmemMax);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_score_stream<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kScoreStreamSmemMax);
+    return e;
+}
+
 // A and B tiles plus 4 KiB of slack after them (never read when the descriptors are right).
 size_t score_umma_smem(int E, int Np) { return (size_t)(kUmmaM + Np) * E * 2 + 4096; }
 
@@ -303,9 +320,6 @@ cudaError_t launch_score(const lsa_dims& d, const SeqTable& tab, int max_n, cons
         uint32_t cols = 32;
         while ((int)cols < Np) cols <<= 1;
         const size_t smem = score_umma_smem(d.E, Np);
-        cudaError_t e = cudaFuncSetAttribute(k_score_umma, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return e;
         cfg.gridDim = dim3((max_n + kUmmaM - 1) / kUmmaM, d.B, 1);
         cfg.blockDim = dim3(128, 1, 1);
         cfg.dynamicSmemBytes = smem;
@@ -324,15 +338,9 @@ cudaError_t launch_score(const lsa_dims& d, const SeqTable& tab, int max_n, cons
     cfg.blockDim = dim3(kScoreThreads, 1, 1);
     cfg.dynamicSmemBytes = (size_t)d.Q * d.E * sizeof(float);
     if (d.emb_dtype == LSA_BF16) {
-        cudaError_t e = cudaFuncSetAttribute(k_score_stream<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)cfg.dynamicSmemBytes);
-        if (e != cudaSuccess) return e;
         return cudaLaunchKernelEx(&cfg, k_score_stream<true>, (const uint8_t*)q_emb,
                                   (const uint8_t*)chunk_emb, scores, tab, d.Q, d.E, rpc);
     }
-    cudaError_t e = cudaFuncSetAttribute(k_score_stream<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)cfg.dynamicSmemBytes);
-    if (e != cudaSuccess) return e;
     return cudaLaunchKernelEx(&cfg, k_score_stream<false>, (const uint8_t*)q_emb,
                               (const uint8_t*)chunk_emb, scores, tab, d.Q, d.E, rpc);
 }

@@ -174,6 +174,12 @@ k_topk(const float* __restrict__ scores, int32_t* __restrict__ ids, const SeqTab
 
 constexpr size_t kTopkSmemKeyLimit = 200 * 1024;
 
+// Raise the dynamic shared-memory limit of the top-k kernel (once per device).
+cudaError_t topk_init_attrs() {
+    return cudaFuncSetAttribute(k_topk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kTopkSmemKeyLimit);
+}
+
 cudaError_t launch_topk(const lsa_dims& d, const SeqTable& tab, int max_n, const float* scores,
                         int32_t* ids, uint32_t* err, cudaStream_t stream, bool pdl) {
     cudaLaunchConfig_t cfg = {};
@@ -187,9 +193,6 @@ cudaError_t launch_topk(const lsa_dims& d, const SeqTable& tab, int max_n, const
     cfg.blockDim = dim3(kTopkThreads, 1, 1);
     const size_t key_bytes = (size_t)max_n * 4;
     if (key_bytes <= kTopkSmemKeyLimit) {
-        cudaError_t e = cudaFuncSetAttribute(k_topk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kTopkSmemKeyLimit);
-        if (e != cudaSuccess) return e;
         cfg.dynamicSmemBytes = key_bytes;
         return cudaLaunchKernelEx(&cfg, k_topk<true>, scores, ids, tab, err);
     }
