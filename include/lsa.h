@@ -146,6 +146,31 @@ LSA_API lsa_status lsa_decode_step(const lsa_dims *dims, const void *q_emb, cons
                            int32_t *chunk_ids_out, float *out, float *lse,
                            void *ws, size_t ws_bytes, void *stream);
 
+/* Sparse decode attention for callers that cannot allocate device memory.
+ * The paper has no counterpart: this is a deployment variant of
+ * lsa_sparse_decode_attn for callers that cannot call cudaMalloc (an engine that
+ * has reserved nearly all device memory for its own pool, a plugin that must not
+ * allocate behind its host framework's allocator, or a latency-critical path where
+ * cudaMalloc's implicit device synchronisation is not acceptable).
+ * Arguments and results are those of lsa_sparse_decode_attn, without a workspace:
+ * the split-K partials live in a fixed LSA_NOALLOC_SCRATCH_BYTES array inside the
+ * library (allocated once per GPU that loads the library, held until exit).
+ *   - Shapes whose partials, (device CTAs + B) * H * (Dh + 2) * 4 bytes plus 256,
+ *     exceed that size are rejected with LSA_ERR_WORKSPACE before any launch.
+ *   - It calls no allocation routine of any kind.
+ *   - The first call on a device (with that device current) looks up the array's
+ *     device address and the device's SM count; make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the array, which keeps the last call's contents;
+ *     each call clears the device error word it uses. Calls whose kernels overlap
+ *     on the GPU race on the array: order them on one stream.
+ *   - Device-side errors (a kept chunk id out of range) are skipped without a fault
+ *     but are not reported: the error word is internal to the library. */
+#define LSA_NOALLOC_SCRATCH_BYTES (4u << 20)
+LSA_API lsa_status lsa_sparse_decode_attn_noalloc(const lsa_dims *dims, const void *q, const void *K,
+                                                  const void *V, const int32_t *chunk_ids, float *out,
+                                                  float *lse, void *stream);
+
 /* Synchronise `stream`, read the sticky device error word of `ws`, clear it, and
  * return LSA_OK or the first device error (NONFINITE, BAD_ID, TIMEOUT, in that order). */
 LSA_API lsa_status lsa_get_device_status(void *ws, void *stream);

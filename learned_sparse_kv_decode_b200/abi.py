@@ -58,6 +58,7 @@ def _load():
         "lsa_sparse_decode_attn": ([dp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "lsa_decode_step": ([dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "lsa_get_device_status": ([vp, vp], ctypes.c_int),
+        "lsa_sparse_decode_attn_noalloc": ([dp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -166,6 +167,13 @@ def lsa_sparse_decode_attn(dims, q, K, V, chunk_ids, out, lse, ws, stream=None) 
 def lsa_decode_step(dims, q_emb, chunk_emb, q, K, V, chunk_ids_out, out, lse, ws, stream=None) -> None:
     _check(lib.lsa_decode_step(dims.ptr, _p(q_emb), _p(chunk_emb), _p(q), _p(K), _p(V), _p(chunk_ids_out),
                                _p(out), _p(lse), _p(ws), _nbytes(ws), _stream(stream)), "lsa_decode_step")
+
+
+def lsa_sparse_decode_attn_noalloc(dims, q, K, V, chunk_ids, out, lse, stream=None) -> None:
+    """lsa_sparse_decode_attn without a workspace, for callers that cannot allocate device
+    memory: the partials live in a fixed scratch array inside the library (see include/lsa.h)."""
+    _check(lib.lsa_sparse_decode_attn_noalloc(dims.ptr, _p(q), _p(K), _p(V), _p(chunk_ids), _p(out), _p(lse),
+                                              _stream(stream)), "lsa_sparse_decode_attn_noalloc")
 
 
 def lsa_get_device_status(ws, stream=None) -> int:
