@@ -25,17 +25,32 @@
 
 namespace lsa {
 
-constexpr int kAttnConsumerWarps = 8;
+// Tunables (compile-time; the defaults are the measured best on B200).
+#ifndef LSA_ATTN_WARPS
+#define LSA_ATTN_WARPS 8        // consumer warps per CTA
+#endif
+#ifndef LSA_ATTN_STAGES
+#define LSA_ATTN_STAGES 3       // ring slots
+#endif
+#ifndef LSA_ATTN_STAGE_BYTES
+#define LSA_ATTN_STAGE_BYTES 32768  // bytes per operand (K or V) per ring slot
+#endif
+
+constexpr int kAttnConsumerWarps = LSA_ATTN_WARPS;
 constexpr int kAttnConsumers = kAttnConsumerWarps * 32;
 constexpr int kAttnThreads = kAttnConsumers + 32;
-constexpr int kStageBytes = 32768;  // per operand (K or V) per ring slot
-constexpr int kStages = 3;
-constexpr int kBatch = 8;           // tokens per online-softmax update
+constexpr int kStageBytes = LSA_ATTN_STAGE_BYTES;
+constexpr int kStages = LSA_ATTN_STAGES;
+// Tokens each consumer group handles per stage when the stage is full-size: a
+// stage holds kStageBytes / (HS*Dh*elem) tokens and a group covers LPH*HS threads,
+// so TOK / TG = kStageBytes / (16 * consumers) for both element sizes.
+constexpr int kTpgMax = kStageBytes / (16 * kAttnConsumers);
+static_assert(kTpgMax >= 1 && (kTpgMax & (kTpgMax - 1)) == 0, "tokens per group must be a power of two");
 
 struct AttnParams {
     int H;                // heads
     int HS;               // heads per CTA (head slice)
-    int TG;               // token groups in a CTA
+    int TG;               // token groups that hold tokens (<= consumers / (LPH * HS))
     int TOK;              // tokens per stage
     int SPC;              // stages per chunk (C / TOK)
     int G;                // CTAs per head slice
@@ -51,7 +66,7 @@ size_t attn_smem_bytes(int lph) {
            (size_t)2 * kStages * 8;
 }
 
-__device__ __forceinline__ int64_t cta_of_stage(int64_t s, int64_t S, int G) {
+__host__ __device__ __forceinline__ int64_t cta_of_stage(int64_t s, int64_t S, int G) {
     return ((s + 1) * G + S - 1) / S - 1;
 }
 
@@ -66,12 +81,28 @@ __device__ __forceinline__ void unpack_vec(const uint4& v, float (&x)[VEC]) {
     }
 }
 
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+// 2^x with the hardware approximation (relative error ~2^-22; 2^-inf = 0).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kAttnConsumers) : "memory");
 }
 
 // grid (G, H / HS), kAttnThreads threads, dynamic smem attn_smem_bytes(LPH).
-template <bool BF16>
+// TPG: tokens per consumer group per stage (TOK / TG).
+template <bool BF16, int TPG>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
              const uint8_t* __restrict__ V, const int32_t* __restrict__ ids,
@@ -86,6 +117,7 @@ k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
     float* scratch = reinterpret_cast<float*>(smem + 2 * kStages * kStageBytes);
     uint64_t* bars = reinterpret_cast<uint64_t*>(scratch + (kAttnConsumers / LPH) * (kDh + 2));
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kStages);
+    __shared__ int s_abort;  // set by a consumer whose bounded wait gave up
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x, hs = blockIdx.y;
@@ -98,6 +130,7 @@ k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
             mbar_init(empty0 + 8 * i, kAttnConsumerWarps);
         }
         fence_mbar_init();
+        s_abort = 0;
     }
     __syncthreads();
     pdl_trigger();
@@ -153,13 +186,11 @@ k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
     const int hl = (tid / LPH) % ap.HS;
     const int tg = tid / (LPH * ap.HS);
     const int h = hs * ap.HS + hl;
-    const int cnt = tg < ap.TOK ? (ap.TOK - tg + ap.TG - 1) / ap.TG : 0;
-    const int cnt_w = __reduce_max_sync(0xffffffffu, cnt);
-    const uint32_t lane_off = (uint32_t)hl * kDh * ES + (uint32_t)li * 16;
+    const bool active = tg < ap.TG;  // warp-uniform: a warp holds whole groups or LPH = 32
+    const uint32_t row = ap.row_bytes;
+    const uint32_t lane_k = smem_u32(sK) + (uint32_t)(tg * TPG) * row + (uint32_t)hl * kDh * ES + li * 16;
+    const uint32_t lane_v = lane_k + kStages * kStageBytes;
 
-    __shared__ int s_abort;  // set by a consumer whose bounded wait gave up
-    if (tid == 0) s_abort = 0;
-    consumer_sync();
     int64_t it = 0;
     bool alive = true;
     int b = seq_of(tab.kept_off, tab.B, s0 / ap.SPC);
@@ -177,7 +208,7 @@ k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
 #pragma unroll
         for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
 
-        for (int64_t s = seg0; s < seg1 && alive; ++s, ++it) {
+        for (int64_t s = seg0; s < seg1; ++s, ++it) {
             const int slot = (int)(it % kStages);
             const uint32_t par = (uint32_t)(it / kStages) & 1u;
             if (!mbar_wait(full0 + 8 * slot, par, err)) {
@@ -185,53 +216,46 @@ k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
                 s_abort = 1;
                 break;
             }
-            const uint8_t* kst = sK + slot * kStageBytes + lane_off;
-            const uint8_t* vst = sV + slot * kStageBytes + lane_off;
-            for (int j0 = 0; j0 < cnt_w; j0 += kBatch) {
-                float sc[kBatch];
+            if (active) {
+                const uint32_t kb = lane_k + slot * kStageBytes;
+                const uint32_t vb = lane_v + slot * kStageBytes;
+                float sc[TPG];
 #pragma unroll
-                for (int j = 0; j < kBatch; ++j) {
-                    const int jj = j0 + j;
-                    sc[j] = 0.f;
-                    if (jj < cnt) {
-                        const int t = tg + jj * ap.TG;
-                        const uint4 kv = *reinterpret_cast<const uint4*>(kst + (uint32_t)t * ap.row_bytes);
-                        float x[VEC];
-                        unpack_vec<BF16, VEC>(kv, x);
+                for (int j = 0; j < TPG; ++j) {
+                    float x[VEC];
+                    unpack_vec<BF16, VEC>(lds128(kb + j * row), x);
+                    float d0 = 0.f, d1 = 0.f;
 #pragma unroll
-                        for (int e = 0; e < VEC; ++e) sc[j] = fmaf(qf[e], x[e], sc[j]);
+                    for (int e = 0; e < VEC; e += 2) {
+                        d0 = fmaf(qf[e], x[e], d0);
+                        d1 = fmaf(qf[e + 1], x[e + 1], d1);
                     }
+                    sc[j] = d0 + d1;
                 }
 #pragma unroll
                 for (int off = LPH / 2; off > 0; off >>= 1) {
 #pragma unroll
-                    for (int j = 0; j < kBatch; ++j) sc[j] += __shfl_xor_sync(0xffffffffu, sc[j], off);
+                    for (int j = 0; j < TPG; ++j) sc[j] += __shfl_xor_sync(0xffffffffu, sc[j], off);
                 }
                 float mx = m;
 #pragma unroll
-                for (int j = 0; j < kBatch; ++j)
-                    if (j0 + j < cnt) mx = fmaxf(mx, sc[j]);
-                const float corr = (mx == -INFINITY) ? 1.f : exp2f(m - mx);
-                float p[kBatch], psum = 0.f;
+                for (int j = 0; j < TPG; ++j) mx = fmaxf(mx, sc[j]);
+                const float corr = ex2(m - mx);
+                float p[TPG], psum = 0.f;
 #pragma unroll
-                for (int j = 0; j < kBatch; ++j) {
-                    p[j] = (j0 + j < cnt) ? exp2f(sc[j] - mx) : 0.f;
+                for (int j = 0; j < TPG; ++j) {
+                    p[j] = ex2(sc[j] - mx);
                     psum += p[j];
                 }
-                l = l * corr + psum;
+                l = fmaf(l, corr, psum);
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) acc[e] *= corr;
 #pragma unroll
-                for (int j = 0; j < kBatch; ++j) {
-                    const int jj = j0 + j;
-                    if (jj < cnt) {
-                        const int t = tg + jj * ap.TG;
-                        const uint4 vv = *reinterpret_cast<const uint4*>(vst + (uint32_t)t * ap.row_bytes);
-                        float x[VEC];
-                        unpack_vec<BF16, VEC>(vv, x);
+                for (int j = 0; j < TPG; ++j) {
+                    float x[VEC];
+                    unpack_vec<BF16, VEC>(lds128(vb + j * row), x);
 #pragma unroll
-                        for (int e = 0; e < VEC; ++e) acc[e] = fmaf(p[j], x[e], acc[e]);
-                    }
+                    for (int e = 0; e < VEC; ++e) acc[e] = fmaf(p[j], x[e], acc[e]);
                 }
                 m = mx;
             }
@@ -244,20 +268,24 @@ k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
         float* po = part_o + ((uint64_t)slot_id * ap.H + h) * kDh + li * VEC;
         float* pml = part_ml + ((uint64_t)slot_id * ap.H + h) * 2;
         if (ap.TG == 1) {
+            if (active) {
 #pragma unroll
-            for (int e = 0; e < VEC; e += 4)
-                *reinterpret_cast<float4*>(po + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
-            if (li == 0) {
-                pml[0] = m;
-                pml[1] = l;
+                for (int e = 0; e < VEC; e += 4)
+                    *reinterpret_cast<float4*>(po + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+                if (li == 0) {
+                    pml[0] = m;
+                    pml[1] = l;
+                }
             }
         } else {
-            float* mine = scratch + (size_t)(tg * ap.HS + hl) * (kDh + 2);
+            if (active) {
+                float* mine = scratch + (size_t)(tg * ap.HS + hl) * (kDh + 2);
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) mine[li * VEC + e] = acc[e];
-            if (li == 0) {
-                mine[kDh] = m;
-                mine[kDh + 1] = l;
+                for (int e = 0; e < VEC; ++e) mine[li * VEC + e] = acc[e];
+                if (li == 0) {
+                    mine[kDh] = m;
+                    mine[kDh + 1] = l;
+                }
             }
             consumer_sync();
             if (tg == 0) {
@@ -268,8 +296,8 @@ k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
                 for (int e = 0; e < VEC; ++e) A[e] = 0.f;
                 for (int g = 0; g < ap.TG; ++g) {
                     const float* o = scratch + (size_t)(g * ap.HS + hl) * (kDh + 2);
-                    const float f = (o[kDh] == -INFINITY) ? 0.f : exp2f(o[kDh] - M);
-                    L += o[kDh + 1] * f;
+                    const float f = ex2(o[kDh] - M);
+                    L = fmaf(o[kDh + 1], f, L);
 #pragma unroll
                     for (int e = 0; e < VEC; ++e) A[e] = fmaf(o[li * VEC + e], f, A[e]);
                 }
@@ -281,42 +309,94 @@ k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
                     pml[1] = L;
                 }
             }
-            consumer_sync();
         }
         seg0 = seg1;
         // every consumer passes the same barriers: leave together if any wait gave up
         consumer_sync();
         if (*(volatile int*)&s_abort) break;
     }
+    (void)alive;
 }
 
-// grid (B, H), 128 threads (one per head-dim element).
-__global__ void __launch_bounds__(kDh)
+// Merge of the split partials of one (sequence, head) with the log-sum-exp rule.
+// grid (B, H, kMergeDimSplit): a CTA merges kMergeDims of the Dh output columns over all of the
+// sequence's slots; kMergeGroups thread groups share the slots so that many loads are in flight.
+constexpr int kMergeDimSplit = 4;
+constexpr int kMergeDims = kDh / kMergeDimSplit;          // 32 columns per CTA
+constexpr int kMergeThreads = 256;
+constexpr int kMergeGroups = kMergeThreads / kMergeDims;  // 8 slot groups
+constexpr int kMergeUnroll = 8;
+constexpr int kMergeMaxSlots = 2048;
+
+__global__ void __launch_bounds__(kMergeThreads)
 k_attn_merge(const float* __restrict__ part_o, const float* __restrict__ part_ml,
              float* __restrict__ out, float* __restrict__ lse, const SeqTable tab,
              const AttnParams ap) {
-    const int b = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
-    const int hs = h / ap.HS;
-    (void)hs;
+    __shared__ float s_w[kMergeMaxSlots];
+    __shared__ float s_red[kMergeThreads / 32];
+    __shared__ float s_acc[kMergeGroups][kMergeDims];
+    const int b = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     pdl_wait();
     const int64_t st0 = (int64_t)tab.kept_off[b] * ap.SPC;
     const int64_t st1 = (int64_t)tab.kept_off[b + 1] * ap.SPC - 1;
-    const int64_t c_lo = cta_of_stage(st0, ap.S, ap.G), c_hi = cta_of_stage(st1, ap.S, ap.G);
-    float M = -INFINITY, L = 0.f, A = 0.f;
-    for (int64_t c = c_lo; c <= c_hi; ++c) {
-        const uint64_t slot = (uint64_t)(c + b);
-        const float m = part_ml[(slot * ap.H + h) * 2];
-        const float l = part_ml[(slot * ap.H + h) * 2 + 1];
-        const float a = part_o[(slot * ap.H + h) * kDh + d];
-        const float Mn = fmaxf(M, m);
-        const float f1 = (M == -INFINITY) ? 0.f : exp2f(M - Mn);
-        const float f2 = (m == -INFINITY) ? 0.f : exp2f(m - Mn);
-        L = L * f1 + l * f2;
-        A = A * f1 + a * f2;
-        M = Mn;
+    const int c_lo = (int)cta_of_stage(st0, ap.S, ap.G);
+    const int ns = (int)cta_of_stage(st1, ap.S, ap.G) - c_lo + 1;
+    const uint64_t slot0 = (uint64_t)c_lo + b;
+
+    // 1. the running maxima m and sums l of all slots -> M
+    float mloc = -INFINITY;
+    for (int i = tid; i < ns; i += kMergeThreads) {
+        const float m = part_ml[((slot0 + i) * ap.H + h) * 2];
+        s_w[i] = m;
+        mloc = fmaxf(mloc, m);
     }
-    out[((uint64_t)b * ap.H + h) * kDh + d] = A / L;
-    if (lse != nullptr && d == 0) lse[(uint64_t)b * ap.H + h] = (M + log2f(L)) * 0.69314718055994531f;
+    for (int off = 16; off > 0; off >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, off));
+    if (lane == 0) s_red[warp] = mloc;
+    __syncthreads();
+    float M = s_red[0];
+#pragma unroll
+    for (int w = 1; w < kMergeThreads / 32; ++w) M = fmaxf(M, s_red[w]);
+    // 2. slot weights 2^(m_s - M) and the merged denominator L
+    float lloc = 0.f;
+    for (int i = tid; i < ns; i += kMergeThreads) {
+        const float w = ex2(s_w[i] - M);
+        s_w[i] = w;
+        lloc = fmaf(part_ml[((slot0 + i) * ap.H + h) * 2 + 1], w, lloc);
+    }
+    for (int off = 16; off > 0; off >>= 1) lloc += __shfl_xor_sync(0xffffffffu, lloc, off);
+    __syncthreads();  // every thread has read s_red (M) before it is reused
+    if (lane == 0) s_red[warp] = lloc;
+    __syncthreads();
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeThreads / 32; ++w) L += s_red[w];
+    // 3. weighted sum of the partial outputs: group g takes slots g, g + groups, ...
+    const int g = tid / kMergeDims, dl = tid % kMergeDims, d = blockIdx.z * kMergeDims + dl;
+    const float* po = part_o + (slot0 * ap.H + h) * kDh + d;
+    const uint64_t sstride = (uint64_t)ap.H * kDh;
+    float a = 0.f;
+    for (int i0 = g; i0 < ns; i0 += kMergeGroups * kMergeUnroll) {
+        float v[kMergeUnroll];
+#pragma unroll
+        for (int u = 0; u < kMergeUnroll; ++u) {
+            const int i = i0 + u * kMergeGroups;
+            v[u] = i < ns ? po[(uint64_t)i * sstride] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kMergeUnroll; ++u) {
+            const int i = i0 + u * kMergeGroups;
+            if (i < ns) a = fmaf(v[u], s_w[i], a);
+        }
+    }
+    s_acc[g][dl] = a;
+    __syncthreads();
+    if (g == 0) {
+        float A = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMergeGroups; ++k) A += s_acc[k][dl];
+        out[((uint64_t)b * ap.H + h) * kDh + d] = A / L;
+        if (lse != nullptr && d == 0) lse[(uint64_t)b * ap.H + h] = (M + log2f(L)) * 0.69314718055994531f;
+    }
 }
 
 // ------------------------------------------------------------------ host side
@@ -324,8 +404,38 @@ struct AttnLaunch {
     AttnParams ap;
     int slices;
     int lph;
+    int tpg;  // tokens per consumer group per stage
     size_t smem;
 };
+
+template <bool BF16, int TPG>
+cudaError_t set_split_attr(size_t smem) {
+    return set_smem_attrs(k_attn_split<BF16, TPG>, (int)smem);
+}
+
+// Every (dtype, tokens-per-group) instantiation the planner can pick.
+template <bool BF16>
+cudaError_t set_split_attrs(size_t smem) {
+    cudaError_t e = set_split_attr<BF16, 1>(smem);
+    if (e == cudaSuccess && kTpgMax >= 2) e = set_split_attr<BF16, (kTpgMax >= 2 ? 2 : 1)>(smem);
+    if (e == cudaSuccess && kTpgMax >= 4) e = set_split_attr<BF16, (kTpgMax >= 4 ? 4 : 1)>(smem);
+    if (e == cudaSuccess && kTpgMax >= 8) e = set_split_attr<BF16, (kTpgMax >= 8 ? 8 : 1)>(smem);
+    return e;
+}
+
+template <bool BF16>
+cudaError_t launch_split(cudaLaunchConfig_t* cfg, int tpg, const void* q, const void* K, const void* V,
+                         const int32_t* ids, float* part_o, float* part_ml, const SeqTable& tab,
+                         const AttnParams& ap, uint32_t* err) {
+    const uint8_t *q8 = (const uint8_t*)q, *K8 = (const uint8_t*)K, *V8 = (const uint8_t*)V;
+    switch (tpg) {
+        case 1: return cudaLaunchKernelEx(cfg, k_attn_split<BF16, 1>, q8, K8, V8, ids, part_o, part_ml, tab, ap, err);
+        case 2: return cudaLaunchKernelEx(cfg, k_attn_split<BF16, (kTpgMax >= 2 ? 2 : 1)>, q8, K8, V8, ids, part_o, part_ml, tab, ap, err);
+        case 4: return cudaLaunchKernelEx(cfg, k_attn_split<BF16, (kTpgMax >= 4 ? 4 : 1)>, q8, K8, V8, ids, part_o, part_ml, tab, ap, err);
+        case 8: return cudaLaunchKernelEx(cfg, k_attn_split<BF16, (kTpgMax >= 8 ? 8 : 1)>, q8, K8, V8, ids, part_o, part_ml, tab, ap, err);
+    }
+    return cudaErrorInvalidValue;
+}
 
 AttnLaunch plan_attention(const lsa_dims& d, const SeqTable& tab, int ctas_per_device, bool indexed) {
     AttnLaunch L = {};
@@ -335,12 +445,14 @@ AttnLaunch plan_attention(const lsa_dims& d, const SeqTable& tab, int ctas_per_d
     AttnParams& ap = L.ap;
     ap.H = d.H;
     ap.HS = d.H < kAttnConsumers / L.lph ? d.H : kAttnConsumers / L.lph;
-    ap.TG = kAttnConsumers / (L.lph * ap.HS);
+    const int groups = kAttnConsumers / (L.lph * ap.HS);
     L.slices = d.H / ap.HS;
     ap.row_bytes = (uint32_t)ap.HS * kDh * es;
     ap.tok_stride = (uint64_t)d.H * kDh * es;
     ap.TOK = kStageBytes / (int)ap.row_bytes;
     if (ap.TOK > d.chunk_len) ap.TOK = d.chunk_len;
+    ap.TG = groups < ap.TOK ? groups : ap.TOK;  // groups beyond the stage's tokens stay idle
+    L.tpg = ap.TOK / ap.TG;
     ap.SPC = d.chunk_len / ap.TOK;
     ap.S = (int64_t)tab.kept_off[d.B] * ap.SPC;
     int G = ctas_per_device / L.slices;
@@ -357,18 +469,17 @@ int attn_max_slots(int ctas_per_device, int B) { return ctas_per_device + B; }
 
 cudaError_t attn_ctas_per_device(lsa_dtype kv, int num_sms, int* out) {
     int occ = 0;
-    cudaError_t e;
+    cudaError_t e = set_smem_attrs(k_attn_merge, 0);
+    if (e != cudaSuccess) return e;
     if (kv == LSA_BF16) {
-        e = cudaFuncSetAttribute(k_attn_split<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)attn_smem_bytes(16));
+        e = set_split_attrs<true>(attn_smem_bytes(16));
         if (e != cudaSuccess) return e;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_attn_split<true>, kAttnThreads,
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_attn_split<true, kTpgMax>, kAttnThreads,
                                                           attn_smem_bytes(16));
     } else {
-        e = cudaFuncSetAttribute(k_attn_split<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)attn_smem_bytes(32));
+        e = set_split_attrs<false>(attn_smem_bytes(32));
         if (e != cudaSuccess) return e;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_attn_split<false>, kAttnThreads,
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_attn_split<false, kTpgMax>, kAttnThreads,
                                                           attn_smem_bytes(32));
     }
     if (e != cudaSuccess) return e;
@@ -393,22 +504,19 @@ cudaError_t launch_attention(const lsa_dims& d, const SeqTable& tab, int ctas_pe
     cfg.gridDim = dim3(L.ap.G, L.slices, 1);
     cfg.blockDim = dim3(kAttnThreads, 1, 1);
     cfg.dynamicSmemBytes = L.smem;
-    cudaError_t e;
-    if (d.kv_dtype == LSA_BF16) {
-        e = cudaLaunchKernelEx(&cfg, k_attn_split<true>, (const uint8_t*)q, (const uint8_t*)K,
-                               (const uint8_t*)V, ids, part_o, part_ml, tab, L.ap, err);
-    } else {
-        e = cudaLaunchKernelEx(&cfg, k_attn_split<false>, (const uint8_t*)q, (const uint8_t*)K,
-                               (const uint8_t*)V, ids, part_o, part_ml, tab, L.ap, err);
-    }
+    if (L.tpg != 1 && L.tpg != 2 && L.tpg != 4 && L.tpg != 8) return cudaErrorInvalidValue;
+    if ((int64_t)L.ap.G > kMergeMaxSlots) return cudaErrorInvalidValue;
+    cudaError_t e = d.kv_dtype == LSA_BF16
+                        ? launch_split<true>(&cfg, L.tpg, q, K, V, ids, part_o, part_ml, tab, L.ap, err)
+                        : launch_split<false>(&cfg, L.tpg, q, K, V, ids, part_o, part_ml, tab, L.ap, err);
     if (e != cudaSuccess) return e;
 
     cudaLaunchConfig_t mcfg = {};
     mcfg.stream = stream;
     mcfg.attrs = attr;
     mcfg.numAttrs = 1;  // the merge always follows the split kernel: overlap its launch
-    mcfg.gridDim = dim3(d.B, d.H, 1);
-    mcfg.blockDim = dim3(kDh, 1, 1);
+    mcfg.gridDim = dim3(d.B, d.H, kMergeDimSplit);
+    mcfg.blockDim = dim3(kMergeThreads, 1, 1);
     mcfg.dynamicSmemBytes = 0;
     return cudaLaunchKernelEx(&mcfg, k_attn_merge, (const float*)part_o, (const float*)part_ml, out,
                               lse, tab, L.ap);

@@ -134,6 +134,19 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
     return p;
 }
 
+// Dynamic shared-memory limit plus the maximum shared-memory carveout, so consecutive
+// kernels of a step do not make the SM switch its L1 / shared-memory split.
+template <typename Kernel>
+inline cudaError_t set_smem_attrs(Kernel* kernel, int max_dynamic_smem) {
+    cudaError_t e = cudaSuccess;
+    if (max_dynamic_smem > 0)
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dynamic_smem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+    return e;
+}
+
 // Sequence of a flattened position `i` given a prefix table (binary search).
 __device__ __forceinline__ int seq_of(const int32_t* off, int B, int64_t i) {
     int lo = 0, hi = B - 1;

@@ -51,16 +51,6 @@ k_score_stream(const uint8_t* __restrict__ q_emb, const uint8_t* __restrict__ em
     const int r1 = min(n_b, r0 + rows_per_cta);
 
     const size_t qbase = (size_t)b * Q * E;
-    for (int i = threadIdx.x; i < Q * E; i += blockDim.x) {
-        if constexpr (BF16) {
-            const uint16_t h = reinterpret_cast<const uint16_t*>(q_emb)[qbase + i];
-            sq[i] = __uint_as_float((uint32_t)h << 16);
-        } else {
-            sq[i] = reinterpret_cast<const float*>(q_emb)[qbase + i];
-        }
-    }
-    __syncthreads();
-
     const int P = E / VEC;            // 16-byte pieces per row
     const int LPR = P < 32 ? P : 32;  // lanes per row
     const int RPW = 32 / LPR;         // rows per warp step
@@ -72,6 +62,60 @@ k_score_stream(const uint8_t* __restrict__ q_emb, const uint8_t* __restrict__ em
     const uint8_t* base = emb + (size_t)tab.chunk_off[b] * row_bytes;
     float* out = scores + tab.chunk_off[b];
     const int step = nwarps * RPW;
+
+    if (Q == 1 && PPL == 1) {
+        // one query, one 16-byte piece per lane: the query piece lives in registers
+        float qv[8];
+        {
+            const uint8_t* qp = q_emb + (qbase + (size_t)li * VEC) * ES;
+            if constexpr (BF16) {
+                unpack16<true>(*reinterpret_cast<const uint4*>(qp), qv);
+            } else {
+                const uint4 t = *reinterpret_cast<const uint4*>(qp);
+                qv[0] = __uint_as_float(t.x); qv[1] = __uint_as_float(t.y);
+                qv[2] = __uint_as_float(t.z); qv[3] = __uint_as_float(t.w);
+            }
+        }
+        for (int wrow = r0 + warp * RPW; wrow < r1; wrow += step * kScoreUnroll) {
+            const int row0 = wrow + sub;
+            uint4 v[kScoreUnroll];
+#pragma unroll
+            for (int u = 0; u < kScoreUnroll; ++u) {
+                const int row = row0 + u * step;
+                v[u] = row < r1 ? ld_stream16(base + (size_t)row * row_bytes + (size_t)li * 16)
+                                : make_uint4(0, 0, 0, 0);
+            }
+            float acc[kScoreUnroll];
+#pragma unroll
+            for (int u = 0; u < kScoreUnroll; ++u) {
+                float x[8];
+                unpack16<BF16>(v[u], x);
+                acc[u] = 0.f;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) acc[u] = fmaf(qv[e], x[e], acc[u]);
+                for (int off = LPR >> 1; off > 0; off >>= 1)
+                    acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], off);
+            }
+            if (li == 0) {
+#pragma unroll
+                for (int u = 0; u < kScoreUnroll; ++u) {
+                    const int row = row0 + u * step;
+                    if (row < r1) out[row] = acc[u];
+                }
+            }
+        }
+        return;
+    }
+
+    for (int i = threadIdx.x; i < Q * E; i += blockDim.x) {
+        if constexpr (BF16) {
+            const uint16_t h = reinterpret_cast<const uint16_t*>(q_emb)[qbase + i];
+            sq[i] = __uint_as_float((uint32_t)h << 16);
+        } else {
+            sq[i] = reinterpret_cast<const float*>(q_emb)[qbase + i];
+        }
+    }
+    __syncthreads();
 
     // The loop bound is warp-uniform (every lane joins the shuffles); rows past r1 are masked.
     for (int wrow = r0 + warp * RPW; wrow < r1; wrow += step * kScoreUnroll) {
@@ -187,38 +231,35 @@ k_score_umma(const uint16_t* __restrict__ q_emb, const uint16_t* __restrict__ em
         fence_mbar_init();
     }
 
-    // ---- stage A (128 chunk rows) and B (Np query rows, zero-padded) into the core-matrix layout
+    // ---- stage A (128 chunk rows) and B (Np query rows, zero-padded) into the core-matrix
+    // layout with asynchronous 16-byte copies (all of a thread's copies in flight at once;
+    // rows past the end are zero-filled without reading global memory)
     const int KC = E / 8;  // 16-byte pieces per row
     const uint16_t* gA = emb + ((size_t)tab.chunk_off[b] + r0) * E;
     const int rows_a = min(kUmmaM, n_b - r0);
     const int pieces_a = kUmmaM * KC;
-    for (int p0 = tid; p0 < pieces_a; p0 += 128 * 4) {
-        uint4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int p = p0 + u * 128;
-            v[u] = make_uint4(0, 0, 0, 0);
-            if (p < pieces_a) {
-                const int r = p & 7, c = (p >> 3) % KC, g = (p >> 3) / KC;
-                const int row = g * 8 + r;
-                if (row < rows_a) v[u] = ld_stream16(gA + (size_t)row * E + c * 8);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int p = p0 + u * 128;
-            if (p < pieces_a) *reinterpret_cast<uint4*>(sA + (size_t)p * 16) = v[u];
-        }
+    const uint32_t sA32 = smem_u32(sA), sB32 = smem_u32(sB);
+    for (int p = tid; p < pieces_a; p += 128) {
+        const int r = p & 7, c = (p >> 3) % KC, g = (p >> 3) / KC;
+        const int row = g * 8 + r;
+        const bool ok = row < rows_a;
+        const uint16_t* src = ok ? gA + (size_t)row * E + c * 8 : gA;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sA32 + p * 16), "l"(src),
+                     "r"(ok ? 16 : 0)
+                     : "memory");
     }
     const uint16_t* gB = q_emb + (size_t)b * Q * E;
     const int pieces_b = Np * KC;
     for (int p = tid; p < pieces_b; p += 128) {
         const int r = p & 7, c = (p >> 3) % KC, g = (p >> 3) / KC;
         const int row = g * 8 + r;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (row < Q) v = *reinterpret_cast<const uint4*>(gB + (size_t)row * E + c * 8);
-        *reinterpret_cast<uint4*>(sB + (size_t)p * 16) = v;
+        const bool ok = row < Q;
+        const uint16_t* src = ok ? gB + (size_t)row * E + c * 8 : gB;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sB32 + p * 16), "l"(src),
+                     "r"(ok ? 16 : 0)
+                     : "memory");
     }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
     // generic-proxy smem writes -> visible to the tensor core (async proxy)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
@@ -286,14 +327,9 @@ k_score_umma(const uint16_t* __restrict__ q_emb, const uint16_t* __restrict__ em
 constexpr int kScoreStreamSmemMax = 200 * 1024;
 size_t score_umma_smem(int E, int Np);
 cudaError_t score_init_attrs() {
-    cudaError_t e = cudaFuncSetAttribute(k_score_umma, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)score_umma_smem(256, 256));
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_score_stream<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kScoreStreamSmemMax);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_score_stream<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kScoreStreamSmemMax);
+    cudaError_t e = set_smem_attrs(k_score_umma, (int)score_umma_smem(256, 256));
+    if (e == cudaSuccess) e = set_smem_attrs(k_score_stream<true>, kScoreStreamSmemMax);
+    if (e == cudaSuccess) e = set_smem_attrs(k_score_stream<false>, kScoreStreamSmemMax);
     return e;
 }
 

@@ -4,17 +4,25 @@
 // step 5): a top-k keep mask over the chunk scores decides which chunks stay
 // resident. Ties go to the lower chunk index; -0.0 and +0.0 are equal.
 //
-// One CTA per sequence runs an exact radix select on order-preserving 32-bit
-// keys (four 8-bit digit passes, most significant first) to find T, the k-th
-// largest key, and how many keys equal to T must be kept. A final pass in index
-// order keeps every key > T plus the lowest-index keys == T, and writes the kept
-// indices in ascending order through a block-wide prefix count (ballots).
+// Exact radix select on order-preserving 32-bit keys, four 8-bit digit passes
+// (most significant first), finding T, the k-th largest key, and how many keys
+// equal to T must be kept. A final pass in index order keeps every key > T plus
+// the lowest-index keys == T and writes the kept indices in ascending order.
+//
+// One sequence runs on a thread-block cluster of CS CTAs (CS = 1..8): CTA r owns
+// a contiguous slice of the sequence's keys (cached in its shared memory). Each
+// pass builds per-CTA digit histograms that every CTA then sums through
+// distributed shared memory (DSMEM); the ordered write uses per-CTA counts
+// exchanged the same way. Cluster barriers are hardware barriers.
 #include "lsa_device.cuh"
 
 namespace lsa {
 
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kTopkMaxCluster = 8;
+constexpr int kTopkKeysPerCta = 2048;  // target slice size when choosing the cluster size
+constexpr size_t kTopkSmemKeyLimit = 192 * 1024;
 
 // Order-preserving map float -> uint32 (larger float -> larger key); -0 maps like +0.
 // NaN maps to 0 (never preferred); NaN and +-Inf set `bad`.
@@ -28,23 +36,54 @@ __device__ __forceinline__ uint32_t score_key(float f, bool& bad) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// grid (B), 1024 threads. SMEM_KEYS: keys cached in dynamic smem (n_max * 4 bytes).
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_size() {
+    uint32_t n;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
+    return n;
+}
+
+// Load a u32 from the shared memory of CTA `rank` of this cluster at the same offset as `p`.
+__device__ __forceinline__ uint32_t dsmem_ld(const uint32_t* p, uint32_t rank) {
+    uint32_t remote, v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(p)), "r"(rank));
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
+    return v;
+}
+
+// grid (CS, B) with cluster (CS, 1, 1), 1024 threads.
+// SMEM_KEYS: the CTA's key slice is cached in dynamic shared memory.
 template <bool SMEM_KEYS>
 __global__ void __launch_bounds__(kTopkThreads)
 k_topk(const float* __restrict__ scores, int32_t* __restrict__ ids, const SeqTable tab,
        uint32_t* err) {
     extern __shared__ uint32_t skeys[];
-    __shared__ uint32_t hist[256];
+    __shared__ uint32_t hist[2][256];  // double-buffered: pass p uses hist[p & 1]
+    __shared__ uint32_t tot[256];
     __shared__ uint32_t s_prefix, s_need;
     __shared__ uint32_t w_gt[kTopkWarps], w_eq[kTopkWarps];
     __shared__ uint32_t o_gt[kTopkWarps], o_eq[kTopkWarps];
     __shared__ uint32_t t_gt, t_eq;
+    __shared__ uint32_t c_gt, c_eq;  // this CTA's totals of keys > T and == T (read by the cluster)
 
-    const int b = blockIdx.x;
+    const int b = blockIdx.y;
+    const uint32_t rank = cluster_rank(), cs = cluster_size();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n = tab.chunk_off[b + 1] - tab.chunk_off[b];
     const int k = tab.kept_off[b + 1] - tab.kept_off[b];
-    const float* s = scores + tab.chunk_off[b];
+    const int slice = (n + (int)cs - 1) / (int)cs;
+    const int lo = min(n, (int)rank * slice), hi = min(n, lo + slice);
+    const int m = hi - lo;  // keys owned by this CTA: indices [lo, hi)
+    const float* s = scores + tab.chunk_off[b] + lo;
     int32_t* out = ids + tab.kept_off[b];
 
     pdl_wait();     // scores come from the preceding kernel
@@ -52,9 +91,9 @@ k_topk(const float* __restrict__ scores, int32_t* __restrict__ ids, const SeqTab
 
     bool bad = false;
     if constexpr (SMEM_KEYS) {
-        for (int i = tid; i < n; i += kTopkThreads) skeys[i] = score_key(s[i], bad);
+        for (int i = tid; i < m; i += kTopkThreads) skeys[i] = score_key(s[i], bad);
     } else {
-        for (int i = tid; i < n; i += kTopkThreads) (void)score_key(s[i], bad);
+        for (int i = tid; i < m; i += kTopkThreads) (void)score_key(s[i], bad);
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(err, kErrNonFinite);
 
@@ -67,26 +106,40 @@ k_topk(const float* __restrict__ scores, int32_t* __restrict__ ids, const SeqTab
         }
     };
 
-    if (tid == 0) {
-        s_prefix = 0;
-        s_need = (uint32_t)k;
-    }
     uint32_t prefix = 0, need = (uint32_t)k;
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
         const uint32_t himask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
-        if (tid < 256) hist[tid] = 0;
+        uint32_t* hp = hist[pass & 1];
+        // hist[pass & 1] was last read two passes ago, before every CTA passed the previous
+        // pass's cluster barrier, so it can be cleared now
+        if (tid < 256) hp[tid] = 0;
         __syncthreads();
-        for (int i0 = 0; i0 < n; i0 += kTopkThreads) {
+        for (int i0 = 0; i0 < m; i0 += kTopkThreads) {
             const int i = i0 + tid;
             uint32_t digit = 256;  // sentinel: not counted
-            if (i < n) {
+            if (i < m) {
                 const uint32_t key = key_at(i);
                 if ((key & himask) == prefix) digit = (key >> shift) & 0xFFu;
             }
             // warp-aggregated histogram update: one atomic per distinct digit in the warp
             const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-            if (digit < 256 && (__ffs(peers) - 1) == lane) atomicAdd(&hist[digit], __popc(peers));
+            if (digit < 256 && (__ffs(peers) - 1) == lane) atomicAdd(&hp[digit], __popc(peers));
+        }
+        if (cs > 1) {
+            cluster_sync_all();  // every CTA's histogram is complete and visible to the cluster
+            if (tid < 256) {
+                uint32_t v[kTopkMaxCluster];
+#pragma unroll
+                for (int r = 0; r < kTopkMaxCluster; ++r) v[r] = (uint32_t)r < cs ? dsmem_ld(&hp[tid], r) : 0u;
+                uint32_t t = 0;
+#pragma unroll
+                for (int r = 0; r < kTopkMaxCluster; ++r) t += v[r];
+                tot[tid] = t;
+            }
+        } else {
+            __syncthreads();
+            if (tid < 256) tot[tid] = hp[tid];
         }
         __syncthreads();
         if (warp == 0) {
@@ -94,7 +147,7 @@ k_topk(const float* __restrict__ scores, int32_t* __restrict__ ids, const SeqTab
             uint32_t h[8], sum = 0;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                h[i] = hist[255 - 8 * lane - i];
+                h[i] = tot[255 - 8 * lane - i];
                 sum += h[i];
             }
             uint32_t incl = sum;
@@ -119,13 +172,53 @@ k_topk(const float* __restrict__ scores, int32_t* __restrict__ ids, const SeqTab
     }
     const uint32_t T = prefix;  // the k-th largest key; keep `need` of the keys equal to T
 
+    // ---- this CTA's counts of keys > T and == T, shared with the cluster
+    {
+        uint32_t g = 0, e = 0;
+        for (int i = tid; i < m; i += kTopkThreads) {
+            const uint32_t key = key_at(i);
+            g += key > T;
+            e += key == T;
+        }
+        g = __reduce_add_sync(0xffffffffu, g);
+        e = __reduce_add_sync(0xffffffffu, e);
+        if (lane == 0) {
+            w_gt[warp] = g;
+            w_eq[warp] = e;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            uint32_t G = 0, E = 0;
+            for (int w = 0; w < kTopkWarps; ++w) {
+                G += w_gt[w];
+                E += w_eq[w];
+            }
+            c_gt = G;
+            c_eq = E;
+        }
+    }
+    uint32_t carry_gt = 0, carry_eq = 0;  // keys > T and == T in lower-ranked CTAs
+    if (cs > 1) {
+        cluster_sync_all();
+        uint32_t vg[kTopkMaxCluster], ve[kTopkMaxCluster];
+#pragma unroll
+        for (int r = 0; r < kTopkMaxCluster; ++r) {
+            vg[r] = (uint32_t)r < rank ? dsmem_ld(&c_gt, r) : 0u;
+            ve[r] = (uint32_t)r < rank ? dsmem_ld(&c_eq, r) : 0u;
+        }
+#pragma unroll
+        for (int r = 0; r < kTopkMaxCluster; ++r) {
+            carry_gt += vg[r];
+            carry_eq += ve[r];
+        }
+    }
+
     // ---- selection in index order
     const uint32_t lt_mask = (1u << lane) - 1u;
-    uint32_t carry_gt = 0, carry_eq = 0;
-    for (int i0 = 0; i0 < n; i0 += kTopkThreads) {
+    for (int i0 = 0; i0 < m; i0 += kTopkThreads) {
         const int i = i0 + tid;
         bool gt = false, eq = false;
-        if (i < n) {
+        if (i < m) {
             const uint32_t key = key_at(i);
             gt = key > T;
             eq = key == T;
@@ -161,37 +254,260 @@ k_topk(const float* __restrict__ scores, int32_t* __restrict__ ids, const SeqTab
         // positions are < k by construction; the bound also guards the output buffer
         if (gt) {
             const uint32_t pos = before_gt + min(before_eq, need);
-            if (pos < (uint32_t)k) out[pos] = i;
+            if (pos < (uint32_t)k) out[pos] = lo + i;
         } else if (eq && before_eq < need) {
             const uint32_t pos = before_gt + before_eq;
-            if (pos < (uint32_t)k) out[pos] = i;
+            if (pos < (uint32_t)k) out[pos] = lo + i;
         }
         carry_gt += t_gt;
         carry_eq += t_eq;
         __syncthreads();
     }
+    if (cs > 1) cluster_sync_all();  // keep this CTA's shared memory alive until the cluster is done reading it
 }
 
-constexpr size_t kTopkSmemKeyLimit = 200 * 1024;
+// ------------------------------------------------------------------ register-resident variant
+// Each of the kTopkRegThreads threads keeps a contiguous run of R keys of its CTA's slice in registers,
+// so the four digit passes and the ordered write need one block barrier each: the digit
+// search runs redundantly in every warp, histograms are triple-buffered (the buffer a pass
+// clears was last read two passes earlier), and the write uses one block-wide scan.
+#ifndef LSA_TOPK_HIST
+#define LSA_TOPK_HIST 1  // histogram update: 0 = warp-aggregated (match.any), 1 = one atomic per key (faster)
+#endif
+#ifndef LSA_TOPK_REG_THREADS
+#define LSA_TOPK_REG_THREADS 256
+#endif
+constexpr int kTopkRegThreads = LSA_TOPK_REG_THREADS;
+constexpr int kTopkRegWarps = kTopkRegThreads / 32;
+
+// Finds the digit d (of 256) where the keys above d number < need <= keys at or above d.
+// Every lane of the calling warp returns the same (digit, keys above d).
+__device__ __forceinline__ void find_digit(const uint32_t* h256, uint32_t need, int lane,
+                                           uint32_t& digit, uint32_t& above_out) {
+    uint32_t h[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        h[i] = h256[255 - 8 * lane - i];
+        sum += h[i];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    uint32_t above = incl - sum;
+    uint32_t found = 0xFFFFFFFFu, fa = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        if (found == 0xFFFFFFFFu && above < need && need <= above + h[i]) {
+            found = (uint32_t)(255 - 8 * lane - i);
+            fa = above;
+        }
+        above += h[i];
+    }
+    const uint32_t who = __ballot_sync(0xffffffffu, found != 0xFFFFFFFFu);
+    const int src = __ffs(who) - 1;  // exactly one lane holds the digit
+    digit = __shfl_sync(0xffffffffu, found, src);
+    above_out = __shfl_sync(0xffffffffu, fa, src);
+}
+
+// grid (CS, B) with cluster (CS, 1, 1), kTopkRegThreads threads; a CTA's slice has at most
+// kTopkRegThreads * R keys.
+template <int R>
+__global__ void __launch_bounds__(kTopkRegThreads)
+k_topk_reg(const float* __restrict__ scores, int32_t* __restrict__ ids, const SeqTable tab,
+           uint32_t* err) {
+    __shared__ uint32_t hist[3][256];
+    __shared__ uint32_t tot[256];
+    __shared__ uint32_t w_gt[kTopkRegWarps], w_eq[kTopkRegWarps];
+    __shared__ uint32_t c_gt, c_eq;  // this CTA's totals of keys > T and == T (read by the cluster)
+
+    const int b = blockIdx.y;
+    const uint32_t rank = cluster_rank(), cs = cluster_size();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n = tab.chunk_off[b + 1] - tab.chunk_off[b];
+    const int k = tab.kept_off[b + 1] - tab.kept_off[b];
+    const int slice = (n + (int)cs - 1) / (int)cs;
+    const int lo = min(n, (int)rank * slice), hi = min(n, lo + slice);
+    const int m = hi - lo;                     // keys of this CTA: [lo, hi)
+    const int base = tid * R;                  // this thread's run: [base, base + R) within the slice
+    const float* s = scores + tab.chunk_off[b] + lo;
+    int32_t* out = ids + tab.kept_off[b];
+
+    if (tid < 256) {
+        hist[0][tid] = 0;
+        hist[1][tid] = 0;
+    }
+    pdl_wait();  // scores come from the preceding kernel
+    pdl_trigger();
+
+    uint32_t kr[R];
+    bool bad = false;
+#pragma unroll
+    for (int j = 0; j < R; ++j) kr[j] = base + j < m ? score_key(s[base + j], bad) : 0u;
+    if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(err, kErrNonFinite);
+    __syncthreads();
+
+    uint32_t prefix = 0, need = (uint32_t)k;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        const uint32_t himask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
+        uint32_t* hp = hist[pass % 3];
+#pragma unroll
+        for (int j = 0; j < R; ++j) {
+            uint32_t digit = 256;
+            if (base + j < m && (kr[j] & himask) == prefix) digit = (kr[j] >> shift) & 0xFFu;
+#if LSA_TOPK_HIST == 0
+            const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+            if (digit < 256 && (__ffs(peers) - 1) == lane) atomicAdd(&hp[digit], __popc(peers));
+#else
+            if (digit < 256) atomicAdd(&hp[digit], 1u);
+#endif
+        }
+        if (tid < 256) hist[(pass + 1) % 3][tid] = 0;  // used next pass; last read two passes ago
+        const uint32_t* h = hp;
+        if (cs > 1) {
+            cluster_sync_all();
+            if (tid < 256) {
+                uint32_t v[kTopkMaxCluster];
+#pragma unroll
+                for (int r = 0; r < kTopkMaxCluster; ++r) v[r] = (uint32_t)r < cs ? dsmem_ld(&hp[tid], r) : 0u;
+                uint32_t t = 0;
+#pragma unroll
+                for (int r = 0; r < kTopkMaxCluster; ++r) t += v[r];
+                tot[tid] = t;
+            }
+            h = tot;
+        }
+        __syncthreads();
+        uint32_t digit, above;
+        find_digit(h, need, lane, digit, above);
+        prefix |= digit << shift;
+        need -= above;
+        if (cs > 1) __syncthreads();  // tot is rewritten by the next pass
+    }
+    const uint32_t T = prefix;  // the k-th largest key; keep `need` of the keys equal to T
+
+    // ---- counts in index order: this thread's run, then a block-wide exclusive scan
+    uint32_t g = 0, e = 0;
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+        if (base + j < m) {
+            g += kr[j] > T;
+            e += kr[j] == T;
+        }
+    }
+    uint32_t ig = g, ie = e;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t vg = __shfl_up_sync(0xffffffffu, ig, off);
+        const uint32_t ve = __shfl_up_sync(0xffffffffu, ie, off);
+        if (lane >= off) {
+            ig += vg;
+            ie += ve;
+        }
+    }
+    if (lane == 31) {
+        w_gt[warp] = ig;
+        w_eq[warp] = ie;
+    }
+    __syncthreads();
+    uint32_t before_g = ig - g, before_e = ie - e, cta_g = 0, cta_e = 0;
+#pragma unroll
+    for (int w = 0; w < kTopkRegWarps; ++w) {
+        const uint32_t a = w_gt[w], c = w_eq[w];
+        if (w < warp) {
+            before_g += a;
+            before_e += c;
+        }
+        cta_g += a;
+        cta_e += c;
+    }
+    if (cs > 1) {
+        if (tid == 0) {
+            c_gt = cta_g;
+            c_eq = cta_e;
+        }
+        cluster_sync_all();
+        uint32_t vg[kTopkMaxCluster], ve[kTopkMaxCluster];
+#pragma unroll
+        for (int r = 0; r < kTopkMaxCluster; ++r) {
+            vg[r] = (uint32_t)r < rank ? dsmem_ld(&c_gt, r) : 0u;
+            ve[r] = (uint32_t)r < rank ? dsmem_ld(&c_eq, r) : 0u;
+        }
+#pragma unroll
+        for (int r = 0; r < kTopkMaxCluster; ++r) {
+            before_g += vg[r];
+            before_e += ve[r];
+        }
+    }
+    // ---- ordered write: every key > T, and the lowest-index `need` keys == T
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+        if (base + j < m) {
+            if (kr[j] > T) {
+                const uint32_t pos = before_g + min(before_e, need);
+                if (pos < (uint32_t)k) out[pos] = lo + base + j;
+                ++before_g;
+            } else if (kr[j] == T) {
+                if (before_e < need) {
+                    const uint32_t pos = before_g + before_e;
+                    if (pos < (uint32_t)k) out[pos] = lo + base + j;
+                }
+                ++before_e;
+            }
+        }
+    }
+    if (cs > 1) cluster_sync_all();  // keep c_gt / c_eq alive until every CTA has read them
+}
 
 // Raise the dynamic shared-memory limit of the top-k kernel (once per device).
 cudaError_t topk_init_attrs() {
-    return cudaFuncSetAttribute(k_topk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)kTopkSmemKeyLimit);
+    cudaError_t e = set_smem_attrs(k_topk<true>, (int)kTopkSmemKeyLimit);
+    if (e == cudaSuccess) e = set_smem_attrs(k_topk<false>, 0);
+    if (e == cudaSuccess) e = set_smem_attrs(k_topk_reg<1>, 0);
+    if (e == cudaSuccess) e = set_smem_attrs(k_topk_reg<2>, 0);
+    if (e == cudaSuccess) e = set_smem_attrs(k_topk_reg<4>, 0);
+    if (e == cudaSuccess) e = set_smem_attrs(k_topk_reg<8>, 0);
+    if (e == cudaSuccess) e = set_smem_attrs(k_topk_reg<16>, 0);
+    return e;
+}
+
+int topk_cluster_size(int max_n) {
+    int cs = 1;
+    while (cs < kTopkMaxCluster && cs * kTopkKeysPerCta < max_n) cs <<= 1;
+    return cs;
 }
 
 cudaError_t launch_topk(const lsa_dims& d, const SeqTable& tab, int max_n, const float* scores,
                         int32_t* ids, uint32_t* err, cudaStream_t stream, bool pdl) {
+    const int cs = topk_cluster_size(max_n);
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.stream = stream;
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    cfg.gridDim = dim3(d.B, 1, 1);
+    cfg.numAttrs = pdl ? 2 : 1;
+    cfg.gridDim = dim3(cs, d.B, 1);
+    const int slice = (max_n + cs - 1) / cs;
+    const int per_thread = (slice + kTopkRegThreads - 1) / kTopkRegThreads;
+    if (per_thread <= 16) {
+        cfg.blockDim = dim3(kTopkRegThreads, 1, 1);
+        cfg.dynamicSmemBytes = 0;
+        if (per_thread <= 1) return cudaLaunchKernelEx(&cfg, k_topk_reg<1>, scores, ids, tab, err);
+        if (per_thread <= 2) return cudaLaunchKernelEx(&cfg, k_topk_reg<2>, scores, ids, tab, err);
+        if (per_thread <= 4) return cudaLaunchKernelEx(&cfg, k_topk_reg<4>, scores, ids, tab, err);
+        if (per_thread <= 8) return cudaLaunchKernelEx(&cfg, k_topk_reg<8>, scores, ids, tab, err);
+        return cudaLaunchKernelEx(&cfg, k_topk_reg<16>, scores, ids, tab, err);
+    }
     cfg.blockDim = dim3(kTopkThreads, 1, 1);
-    const size_t key_bytes = (size_t)max_n * 4;
+    const size_t key_bytes = (size_t)slice * 4;
     if (key_bytes <= kTopkSmemKeyLimit) {
         cfg.dynamicSmemBytes = key_bytes;
         return cudaLaunchKernelEx(&cfg, k_topk<true>, scores, ids, tab, err);

@@ -85,7 +85,9 @@ def _tie_scores(n, seed, levels=4.0):
 
 
 @pytest.mark.parametrize("N,k", [((1,), (1,)), ((7, 64), (3, 64)), ((1000, 999), (1, 998)),
-                                 ((5000, 16384), (700, 2212)), ((60000,), (6000,))])
+                                 ((5000, 16384), (700, 2212)), ((60000,), (6000,)),
+                                 ((120_000,), (16_000,)),       # per-CTA slices in shared memory
+                                 ((400_000, 3), (54_000, 2))])  # slices too big for shared memory
 def test_topk_bit_exact_with_ties(lsa, N, k):
     w = datagen.small_workload(B=len(N), N=N, k=k, E=64)
     dims = G.dims_of(w, lsa)
