@@ -43,7 +43,7 @@ def parse_args():
     p.add_argument("--steps", type=int, default=5000)
     p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="128k", choices=["tiny", "128k", "128k-b2", "500k", "1m", "mixed"])
+    p.add_argument("--workload", default="128k", choices=["tiny", "128k", "128k-b2", "500k", "1m", "1m-h2", "mixed"])
     p.add_argument("--contexts", default="500k,1m",
                    help="extra workloads timed in the same run (comma list, '' for none)")
     p.add_argument("--rotations", type=int, default=4, help="distinct query sets cycled over the steps")

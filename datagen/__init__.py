@@ -222,6 +222,9 @@ def workload(name: str) -> Workload:
     if name == "1m":
         return Workload("1m", 1, [16384], 256, 64, [2212], 16, seed=3, plant="copy_query",
                         plant_count=[164])
+    if name == "1m-h2":  # the 1M lookahead shape with 2 heads: a profiling case (1.1 GB of K/V)
+        return Workload("1m-h2", 1, [16384], 256, 64, [2212], 2, seed=3, plant="copy_query",
+                        plant_count=[164])
     if name == "mixed":
         L = _mixed_lengths(4, 32)
         N = [l // 64 for l in L]

@@ -16,6 +16,9 @@
 //  * k_score_umma   - Q > 1 with bf16 embeddings: a tcgen05 tensor-core GEMM,
 //    D[128 x Qp] = A[128 chunks x E] * B[Qp queries x E]^T accumulated in TMEM,
 //    followed by a per-row max in the epilogue (tcgen05.ld).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "lsa_device.cuh"
 
 namespace lsa {
@@ -166,11 +169,11 @@ k_score_stream(const uint8_t* __restrict__ q_emb, const uint8_t* __restrict__ em
 }
 
 // ============================================================== tcgen05 GEMM + row max
-// Shared-memory operand layout: K-major, no swizzle ("interleaved" canonical
-// layout). An 8-row x 16-byte core matrix is 128 contiguous bytes; core
-// matrices adjacent along K are LBO = 128 bytes apart, and 8-row groups are
-// SBO = E*16 bytes apart. Piece p = ((g*KC + c)*8 + r) sits at byte p*16, so a
-// warp's 16-byte stores are contiguous.
+// Shared-memory operand layout: K-major, no swizzle ("interleaved" canonical layout),
+// written directly by 2-D TMA tile loads. The tile of K-chunk c (8 bf16 = 16 bytes of
+// every row) is one box of [rows x 16 bytes], stored rows-contiguous, so an 8-row x
+// 16-byte core matrix is 128 contiguous bytes, 8-row groups are SBO = 128 bytes apart
+// and K-chunks are LBO = rows * 16 bytes apart.
 __device__ __forceinline__ uint64_t umma_desc_k_noswizzle(uint32_t saddr, uint32_t lbo,
                                                           uint32_t sbo) {
     uint64_t d = 0;
@@ -198,14 +201,26 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// 2-D TMA tile load (no multicast) of the box at (x = column, y = row) into shared memory.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
 constexpr int kUmmaM = 128;
 
 // grid (ceil(maxN/128), B), 128 threads; dynamic smem: A (128*E*2) + B (Np*E*2), 1 KiB aligned.
+// tmA: chunk embeddings [sum N][E] bf16, box 8 x 128; tmB: query embeddings [B*Q][E], box 8 x Np.
 __global__ void __launch_bounds__(128)
-k_score_umma(const uint16_t* __restrict__ q_emb, const uint16_t* __restrict__ emb,
+k_score_umma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
              float* __restrict__ scores, const SeqTable tab, int Q, int Np, int E,
              uint32_t tmem_cols, uint32_t* err) {
     extern __shared__ __align__(1024) uint8_t smem[];
+    __shared__ __align__(8) uint64_t load_bar;
     __shared__ __align__(8) uint64_t mma_bar;
     __shared__ uint32_t tmem_slot;
 
@@ -215,10 +230,16 @@ k_score_umma(const uint16_t* __restrict__ q_emb, const uint16_t* __restrict__ em
     pdl_trigger();
     if (r0 >= n_b) return;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int KC = E / 8;  // 16-byte K-chunks per row
+    const uint32_t sA = smem_u32(smem), sB = sA + (uint32_t)kUmmaM * E * 2;
 
-    uint8_t* sA = smem;
-    uint8_t* sB = smem + (size_t)kUmmaM * E * 2;
-
+    if (tid == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+        mbar_init(smem_u32(&load_bar), 1);
+        mbar_init(smem_u32(&mma_bar), 1);
+        fence_mbar_init();
+    }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(&tmem_slot)),
@@ -226,73 +247,52 @@ k_score_umma(const uint16_t* __restrict__ q_emb, const uint16_t* __restrict__ em
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    if (tid == 0) {
-        mbar_init(smem_u32(&mma_bar), 1);
-        fence_mbar_init();
-    }
-
-    // ---- stage A (128 chunk rows) and B (Np query rows, zero-padded) into the core-matrix
-    // layout with asynchronous 16-byte copies (all of a thread's copies in flight at once;
-    // rows past the end are zero-filled without reading global memory)
-    const int KC = E / 8;  // 16-byte pieces per row
-    const uint16_t* gA = emb + ((size_t)tab.chunk_off[b] + r0) * E;
-    const int rows_a = min(kUmmaM, n_b - r0);
-    const int pieces_a = kUmmaM * KC;
-    const uint32_t sA32 = smem_u32(sA), sB32 = smem_u32(sB);
-    for (int p = tid; p < pieces_a; p += 128) {
-        const int r = p & 7, c = (p >> 3) % KC, g = (p >> 3) / KC;
-        const int row = g * 8 + r;
-        const bool ok = row < rows_a;
-        const uint16_t* src = ok ? gA + (size_t)row * E + c * 8 : gA;
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sA32 + p * 16), "l"(src),
-                     "r"(ok ? 16 : 0)
-                     : "memory");
-    }
-    const uint16_t* gB = q_emb + (size_t)b * Q * E;
-    const int pieces_b = Np * KC;
-    for (int p = tid; p < pieces_b; p += 128) {
-        const int r = p & 7, c = (p >> 3) % KC, g = (p >> 3) / KC;
-        const int row = g * 8 + r;
-        const bool ok = row < Q;
-        const uint16_t* src = ok ? gB + (size_t)row * E + c * 8 : gB;
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sB32 + p * 16), "l"(src),
-                     "r"(ok ? 16 : 0)
-                     : "memory");
-    }
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-    // generic-proxy smem writes -> visible to the tensor core (async proxy)
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_d = tmem_slot;
 
+    bool loaded = true;
     if (tid == 0) {
-        const uint32_t idesc = umma_idesc_bf16_f32(kUmmaM, Np);
-        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
-        const uint32_t sbo = (uint32_t)E * 16;
-        for (int ks = 0; ks < E / 16; ++ks) {
-            const uint64_t ad = umma_desc_k_noswizzle(a0 + ks * 256, 128, sbo);
-            const uint64_t bd = umma_desc_k_noswizzle(b0 + ks * 256, 128, sbo);
-            const uint32_t accum = ks > 0 ? 1u : 0u;
-            asm volatile(
-                "{\n\t.reg .pred p;\n\t"
-                "setp.ne.b32 p, %4, 0;\n\t"
-                "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-                "l"(ad), "l"(bd), "r"(idesc), "r"(accum)
-                : "memory");
+        // one thread stages both operands; rows past the tensor read as zeros, rows of the next
+        // sequence (inside the tensor) are loaded and masked in the epilogue
+        const uint32_t lb = smem_u32(&load_bar);
+        mbar_arrive_expect_tx(lb, (uint32_t)(kUmmaM + Np) * E * 2);
+        const int rowA = tab.chunk_off[b] + r0, rowB = b * Q;
+        for (int c = 0; c < KC; ++c) {
+            tma_load_2d(sA + (uint32_t)c * kUmmaM * 16, &tmA, c * 8, rowA, lb);
+            tma_load_2d(sB + (uint32_t)c * Np * 16, &tmB, c * 8, rowB, lb);
         }
-        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                         smem_u32(&mma_bar))
-                     : "memory");
+        loaded = mbar_wait(lb, 0, err);
+        if (loaded) {
+            const uint32_t idesc = umma_idesc_bf16_f32(kUmmaM, Np);
+            for (int ks = 0; ks < E / 16; ++ks) {
+                // K-step ks covers K-chunks 2ks and 2ks+1
+                const uint64_t ad = umma_desc_k_noswizzle(sA + (uint32_t)ks * 2 * kUmmaM * 16, kUmmaM * 16, 128);
+                const uint64_t bd = umma_desc_k_noswizzle(sB + (uint32_t)ks * 2 * Np * 16, (uint32_t)Np * 16, 128);
+                const uint32_t accum = ks > 0 ? 1u : 0u;
+                asm volatile(
+                    "{\n\t.reg .pred p;\n\t"
+                    "setp.ne.b32 p, %4, 0;\n\t"
+                    "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+                    "l"(ad), "l"(bd), "r"(idesc), "r"(accum)
+                    : "memory");
+            }
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                             smem_u32(&mma_bar))
+                         : "memory");
+        } else {
+            mbar_arrive(smem_u32(&mma_bar));  // no MMA was issued: release the waiters
+        }
     }
     // warp-uniform: the tcgen05.ld below is .sync.aligned
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&mma_bar), 0, err));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&mma_bar), 0, err) && loaded);
+    const bool all_ok = __syncthreads_and(ok);
     tc_fence_after();
 
     // ---- epilogue: row r0 + 32*warp + lane lives in TMEM lane 32*warp + lane
     float best = -INFINITY;
-    if (ok) {
+    if (all_ok) {
         const uint32_t taddr = tmem_d + ((uint32_t)(warp * 32) << 16);
         for (int c0 = 0; c0 < Np; c0 += 16) {
             uint32_t r[16];
@@ -318,6 +318,28 @@ k_score_umma(const uint16_t* __restrict__ q_emb, const uint16_t* __restrict__ em
                      "r"(tmem_cols)
                      : "memory");
     }
+}
+
+// Host: a 2-D tensor map over a row-major bf16 matrix [rows][cols] with a box of
+// [box_rows x 8 columns] (16 bytes per row), no swizzle, zero fill outside the tensor.
+cudaError_t make_tmap_rows16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                             uint32_t box_rows) {
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (encode == nullptr) {
+        cudaDriverEntryPointQueryResult q;
+        void* fn = nullptr;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr) return cudaErrorInvalidValue;
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {8, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 // ============================================================== launchers
@@ -355,12 +377,14 @@ cudaError_t launch_score(const lsa_dims& d, const SeqTable& tab, int max_n, cons
         const int Np = (d.Q + 15) / 16 * 16;
         uint32_t cols = 32;
         while ((int)cols < Np) cols <<= 1;
-        const size_t smem = score_umma_smem(d.E, Np);
+        CUtensorMap tmA, tmB;
+        cudaError_t e = make_tmap_rows16(&tmA, chunk_emb, (uint64_t)tab.chunk_off[d.B], d.E, kUmmaM);
+        if (e == cudaSuccess) e = make_tmap_rows16(&tmB, q_emb, (uint64_t)d.B * d.Q, d.E, (uint32_t)Np);
+        if (e != cudaSuccess) return e;
         cfg.gridDim = dim3((max_n + kUmmaM - 1) / kUmmaM, d.B, 1);
         cfg.blockDim = dim3(128, 1, 1);
-        cfg.dynamicSmemBytes = smem;
-        return cudaLaunchKernelEx(&cfg, k_score_umma, (const uint16_t*)q_emb,
-                                  (const uint16_t*)chunk_emb, scores, tab, d.Q, Np, d.E, cols, err);
+        cfg.dynamicSmemBytes = score_umma_smem(d.E, Np);
+        return cudaLaunchKernelEx(&cfg, k_score_umma, tmA, tmB, scores, tab, d.Q, Np, d.E, cols, err);
     }
     const int es = d.emb_dtype == LSA_BF16 ? 2 : 4;
     const int P = d.E * es / 16;
