@@ -390,6 +390,9 @@ def run_ours(args):
             res["attn_ms"] = ams / K
             # end to end through the public call with host buffers: H2D queries, step, D2H results
             res["e2e"] = e2e_loop(S, K, W, world)
+            # the pages' retrieval interval: re-score and refresh the resident set every 64 steps,
+            # attend over the resident buffer in between (an extra mode, not the headline)
+            res["interval64"] = interval_loop(S, K, W, world)
         results[name] = res
         if name != args.workload:
             del S
@@ -487,6 +490,52 @@ def e2e_loop(S, K: int, W: int, world: int) -> dict:
     bo = h_out.numel() * h_out.element_size() + h_ids.numel() * h_ids.element_size()
     return {"value": K / (ms / 1e3) * world, "unit": "steps/s", "h2d_bytes_per_step": bi,
             "d2h_bytes_per_step": bo, "ms_per_step": ms / K}
+
+
+def interval_loop(S, K: int, W: int, world: int, every: int = 64) -> dict:
+    """Steps/s of the lookahead loop: one retrieval cycle (score, top-k, incremental resident
+    refresh) every `every` steps, attention over the resident buffer at every step."""
+    import torch
+    w, lsa = S.w, S.lsa
+    R = len(S.q)
+    tdt = S.K.dtype
+    slots = torch.full((w.total_kept,), -1, dtype=torch.int32, device="cuda")
+    K_res = torch.empty((w.total_kept * w.C, w.H, w.Dh), dtype=tdt, device="cuda")
+    V_res = torch.empty_like(K_res)
+    moved = torch.zeros(w.B, dtype=torch.int32, device="cuda")
+
+    def cycle(r):
+        lsa.lsa_refresh_resident(S.dims, S.q_emb[r], S.chunk_emb, S.K, S.V, slots, K_res, V_res, moved, S.ws)
+        for i in range(every):
+            lsa.lsa_sparse_decode_attn(S.dims, S.q[(r + i) % R], K_res, V_res, None, S.out, S.lse, S.ws)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for r in range(R):
+            cycle(r)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graphs = []
+    for r in range(R):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            cycle(r)
+        graphs.append(g)
+    cycles = max(1, K // every)
+    ms = time_loop(lambda i: graphs[i % R].replay(), cycles, max(1, W // every) + 1, world)
+    moved_per_cycle = int(moved.sum().item())
+    st = lsa.lsa_get_device_status(S.ws)
+    if st != lsa.LSA_OK:
+        raise SystemExit(f"device error in the interval loop: {lsa.string(st)}")
+    kv = w.esize("kv_dtype")
+    chunk_bytes = w.C * w.H * w.Dh * kv
+    cycle_bytes = (w.total_chunks * w.E * w.esize("emb_dtype") + moved_per_cycle * chunk_bytes * 4
+                   + every * (w.total_kept * chunk_bytes * 2 + w.B * w.H * w.Dh * (kv + 4)))
+    steps = cycles * every
+    return {"every": every, "steps": steps, "steps_per_s": steps / (ms / 1e3) * world,
+            "ms_per_step": ms / steps, "moved_chunks_per_cycle": moved_per_cycle,
+            "gbs": cycle_bytes * cycles / (ms / 1e3) / 1e9 * world}
 
 
 def main():

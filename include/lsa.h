@@ -146,6 +146,23 @@ LSA_API lsa_status lsa_decode_step(const lsa_dims *dims, const void *q_emb, cons
                            int32_t *chunk_ids_out, float *out, float *lse,
                            void *ws, size_t ws_bytes, void *stream);
 
+/* Retrieval cycle of the lookahead loop [R3-2.3 steps 4-7; review section 3-1: the
+ * indexer re-scores about every 64 decode steps and attention runs over the kept
+ * chunks until the next cycle]. Scores every chunk, keeps the top-k, and refreshes a
+ * resident buffer so that it holds exactly the kept chunks, copying only entering ones.
+ *   slot_ids     [sum k_b] int32, in/out: slot j of sequence b holds local chunk
+ *                slot_ids[kept_off_b + j], or is empty (-1; fill with -1 for a cold start).
+ *                Chunks that stay keep their slot; entering chunks (ascending) fill the freed
+ *                slots (ascending). A chunk listed twice stays in one of its slots only.
+ *   K_res, V_res [sum k_b * C][H][Dh] kv_dtype, in/out: slot j = rows [(kept_off_b+j)*C, +C).
+ *   moved        [B] int32 device, out, or NULL: chunks copied per sequence.
+ * Per-step attention between cycles: lsa_sparse_decode_attn with chunk_ids = NULL over
+ * K_res/V_res (the slot order does not change the softmax). Requires N_b <= 2^19. */
+LSA_API lsa_status lsa_refresh_resident(const lsa_dims *dims, const void *q_emb, const void *chunk_emb,
+                                        const void *K, const void *V, int32_t *slot_ids, void *K_res,
+                                        void *V_res, int32_t *moved, void *ws, size_t ws_bytes,
+                                        void *stream);
+
 /* Sparse decode attention for callers that cannot allocate device memory.
  * The paper has no counterpart: this is a deployment variant of
  * lsa_sparse_decode_attn for callers that cannot call cudaMalloc (an engine that

@@ -59,6 +59,7 @@ def _load():
         "lsa_decode_step": ([dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "lsa_get_device_status": ([vp, vp], ctypes.c_int),
         "lsa_sparse_decode_attn_noalloc": ([dp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+        "lsa_refresh_resident": ([dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -167,6 +168,12 @@ def lsa_sparse_decode_attn(dims, q, K, V, chunk_ids, out, lse, ws, stream=None) 
 def lsa_decode_step(dims, q_emb, chunk_emb, q, K, V, chunk_ids_out, out, lse, ws, stream=None) -> None:
     _check(lib.lsa_decode_step(dims.ptr, _p(q_emb), _p(chunk_emb), _p(q), _p(K), _p(V), _p(chunk_ids_out),
                                _p(out), _p(lse), _p(ws), _nbytes(ws), _stream(stream)), "lsa_decode_step")
+
+
+def lsa_refresh_resident(dims, q_emb, chunk_emb, K, V, slot_ids, K_res, V_res, moved, ws, stream=None) -> None:
+    _check(lib.lsa_refresh_resident(dims.ptr, _p(q_emb), _p(chunk_emb), _p(K), _p(V), _p(slot_ids), _p(K_res),
+                                    _p(V_res), _p(moved), _p(ws), _nbytes(ws), _stream(stream)),
+           "lsa_refresh_resident")
 
 
 def lsa_sparse_decode_attn_noalloc(dims, q, K, V, chunk_ids, out, lse, stream=None) -> None:

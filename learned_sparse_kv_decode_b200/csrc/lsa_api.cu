@@ -21,6 +21,12 @@ cudaError_t launch_gather(const lsa_dims& d, const SeqTable& tab, const void* K,
 cudaError_t attn_ctas_per_device(lsa_dtype kv, int num_sms, int* out);
 cudaError_t score_init_attrs();
 cudaError_t topk_init_attrs();
+cudaError_t refresh_init_attrs();
+int refresh_max_chunks();
+cudaError_t launch_refresh(const lsa_dims& d, const SeqTable& tab, int max_n, const int32_t* new_ids,
+                           int32_t* slot_ids, const void* K, const void* V, void* K_res, void* V_res,
+                           int32_t* copy_src, int32_t* copy_dst, int32_t* copy_count, int32_t* moved,
+                           cudaStream_t stream);
 cudaError_t launch_attention(const lsa_dims& d, const SeqTable& tab, int ctas_per_device,
                              const void* q, const void* K, const void* V, const int32_t* ids,
                              float* part_o, float* part_ml, float* out, float* lse, uint32_t* err,
@@ -53,7 +59,9 @@ lsa_status device_info(DeviceInfo* out) {
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return LSA_ERR_CUDA;
         di.sms = sms;
         // kernel attributes are per device: set them here, never inside a launch (graph capture)
-        if (score_init_attrs() != cudaSuccess || topk_init_attrs() != cudaSuccess) return LSA_ERR_CUDA;
+        if (score_init_attrs() != cudaSuccess || topk_init_attrs() != cudaSuccess ||
+            refresh_init_attrs() != cudaSuccess)
+            return LSA_ERR_CUDA;
         if (attn_ctas_per_device(LSA_F32, sms, &di.attn_ctas[LSA_F32]) != cudaSuccess) return LSA_ERR_CUDA;
         if (attn_ctas_per_device(LSA_BF16, sms, &di.attn_ctas[LSA_BF16]) != cudaSuccess) return LSA_ERR_CUDA;
         di.ready = true;
@@ -122,16 +130,21 @@ lsa_status prepare(const lsa_dims* d, Prepared* p) {
 }
 
 struct WsLayout {
-    size_t scores, part_o, part_ml, total;
+    size_t scores, part_o, part_ml, ids, copy_src, copy_dst, copy_count, total;
 };
 
+// Workspace: header (sticky error word) | scores | split partials | refresh buffers.
 WsLayout ws_layout(const lsa_dims* d, const Prepared& p, const DeviceInfo& di) {
     WsLayout w;
     const int slots = di.attn_ctas[d->kv_dtype] + d->B;
     w.scores = kWsHeader;
     w.part_o = align256(w.scores + (size_t)p.total_chunks * 4);
     w.part_ml = align256(w.part_o + (size_t)slots * d->H * LSA_HEAD_DIM * 4);
-    w.total = align256(w.part_ml + (size_t)slots * d->H * 2 * 4);
+    w.ids = align256(w.part_ml + (size_t)slots * d->H * 2 * 4);
+    w.copy_src = align256(w.ids + (size_t)p.total_kept * 4);
+    w.copy_dst = align256(w.copy_src + (size_t)p.total_kept * 4);
+    w.copy_count = align256(w.copy_dst + (size_t)p.total_kept * 4);
+    w.total = align256(w.copy_count + (size_t)d->B * 4);
     return w;
 }
 
@@ -267,6 +280,33 @@ lsa_status lsa_decode_step(const lsa_dims* dims, const void* q_emb, const void* 
     e = launch_attention(*dims, p.tab, di.attn_ctas[dims->kv_dtype], q, K, V, chunk_ids_out,
                          reinterpret_cast<float*>(at(ws, w.part_o)),
                          reinterpret_cast<float*>(at(ws, w.part_ml)), out, lse, err, st, true);
+    return cuda_status(e);
+}
+
+lsa_status lsa_refresh_resident(const lsa_dims* dims, const void* q_emb, const void* chunk_emb,
+                                const void* K, const void* V, int32_t* slot_ids, void* K_res,
+                                void* V_res, int32_t* moved, void* ws, size_t ws_bytes, void* stream) {
+    Prepared p;
+    DeviceInfo di;
+    WsLayout w;
+    lsa_status s = prepare_ws(dims, ws, ws_bytes, &p, &di, &w);
+    if (s != LSA_OK) return s;
+    if (!aligned16(q_emb) || !aligned16(chunk_emb) || !aligned16(K) || !aligned16(V) ||
+        !aligned16(slot_ids) || !aligned16(K_res) || !aligned16(V_res))
+        return LSA_ERR_INVALID_ARG;
+    if (moved != nullptr && (reinterpret_cast<uintptr_t>(moved) & 3u)) return LSA_ERR_INVALID_ARG;
+    if (p.max_n > refresh_max_chunks()) return LSA_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+    float* scores = reinterpret_cast<float*>(at(ws, w.scores));
+    int32_t* ids = reinterpret_cast<int32_t*>(at(ws, w.ids));
+    cudaError_t e = launch_score(*dims, p.tab, p.max_n, q_emb, chunk_emb, scores, err, di.sms, st, false);
+    if (e == cudaSuccess) e = launch_topk(*dims, p.tab, p.max_n, scores, ids, err, st, true);
+    if (e == cudaSuccess)
+        e = launch_refresh(*dims, p.tab, p.max_n, ids, slot_ids, K, V, K_res, V_res,
+                           reinterpret_cast<int32_t*>(at(ws, w.copy_src)),
+                           reinterpret_cast<int32_t*>(at(ws, w.copy_dst)),
+                           reinterpret_cast<int32_t*>(at(ws, w.copy_count)), moved, st);
     return cuda_status(e);
 }
 

@@ -15,7 +15,9 @@ dimensionstp.github.io, section 3-2 (2)-(3); arXiv abstract):
 3. gather: the kept chunks' K/V rows, in kept order (a compaction);
 4. exact softmax attention of the decode query over the kept tokens only,
    scale 1/sqrt(Dh), returning the output and the log-sum-exp per head;
-5. footprint = k * chunk_len / L.
+5. footprint = k * chunk_len / L;
+6. the retrieval cycle's resident refresh (review section 3-1 "retrieval interval" and
+   section 3-2 (3) step 7): the slot table after a cycle, written out as its rule.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (hand-worked fixtures in ``tests/golden/``, closed forms, a brute-force
@@ -130,3 +132,32 @@ def decode_step(q_emb, chunk_emb, q, K, V, k: int, chunk_len: int, scale: float 
     Vk = V(tok) if callable(V) else np.asarray(V)[tok]
     out, lse = attention(q, Kk, Vk, scale)
     return ids, out, lse, s
+
+
+def refresh_resident(old_slots, new_ids, n: int):
+    """Resident slot table after a retrieval cycle, and the copies it needs.
+
+    Review of FlashMemory-DeepSeek-V4, section 3-1 (re-score about every 64 decode
+    steps) and section 3-2 (3) step 7 (attend over the kept chunks until the next
+    cycle); only the kept chunks stay resident (abstract). The rule: a slot whose chunk
+    (valid, 0 <= c < n) is still kept keeps it (a chunk listed twice stays in its first
+    slot); every other slot is freed; the entering chunks in ascending order fill the
+    freed slots in ascending order. Returns (slots, copies) with copies a list of
+    (chunk, slot) pairs, the only chunks whose rows move."""
+    new = sorted(int(c) for c in new_ids)
+    new_set = set(new)
+    slots = [int(c) for c in old_slots]
+    staying = set()
+    freed = []
+    for j, c in enumerate(slots):
+        if 0 <= c < n and c in new_set and c not in staying:
+            staying.add(c)
+        else:
+            freed.append(j)
+    entering = [c for c in new if c not in staying]
+    assert len(entering) == len(freed)
+    copies = []
+    for c, j in zip(entering, freed):
+        slots[j] = c
+        copies.append((c, j))
+    return np.array(slots, dtype=np.int32), copies

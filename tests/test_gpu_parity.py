@@ -323,3 +323,97 @@ def test_argument_errors(lsa):
     with pytest.raises(lsa.LsaError) as e:
         lsa.lsa_sparse_decode_attn(dw.dims, None, dw.K, dw.V, dw.ids, dw.out, None, dw.ws)
     assert e.value.status == lsa.LSA_ERR_INVALID_ARG
+
+
+# ------------------------------------------------------------------ resident refresh (retrieval cycle)
+REFRESH_CASES = [
+    dict(B=2, N=(40, 72), k=(6, 11), E=64, H=8, kv_dtype="f32", emb_dtype="f32"),
+    dict(B=3, N=(300, 129, 64), k=(40, 17, 64), E=128, H=16, kv_dtype="bf16", emb_dtype="bf16"),
+    dict(B=1, N=(600,), k=(81,), E=256, Q=64, H=16, kv_dtype="bf16", emb_dtype="bf16", plant="copy_query"),
+]
+
+
+def _check_resident(dw, slots, Kr, Vr, skip=None):
+    w = dw.w
+    Kg, Vg = Kr.float().cpu().numpy(), Vr.float().cpu().numpy()
+    for b in range(w.B):
+        for j in range(w.k[b]):
+            g = int(w.k_offsets[b]) + j
+            if skip is not None and g in skip:
+                continue
+            tok = oracle.kept_tokens([slots[g]], w.C)
+            rows = slice(g * w.C, (g + 1) * w.C)
+            np.testing.assert_array_equal(Kg[rows], dw.kv_f("K", b, tok))
+            np.testing.assert_array_equal(Vg[rows], dw.kv_f("V", b, tok))
+
+
+@pytest.mark.parametrize("case", REFRESH_CASES, ids=lambda c: f"B{c['B']}-Q{c.get('Q', 1)}-{c['kv_dtype']}")
+def test_refresh_resident_cycles(lsa, case):
+    w = datagen.small_workload(seed=55, **case)
+    dw = G.DeviceWorkload(w, lsa)
+    koff = w.k_offsets
+    slots = torch.full((w.total_kept,), -1, dtype=torch.int32, device="cuda")
+    Kr = torch.zeros((w.total_kept * w.C, w.H, w.Dh), dtype=G.tdtype(w.kv_dtype), device="cuda")
+    Vr = torch.zeros_like(Kr)
+    moved = torch.zeros(w.B, dtype=torch.int32, device="cuda")
+
+    def oracle_ids(q_emb_host):
+        out = []
+        for b in range(w.B):
+            qf = datagen.as_f32(q_emb_host[b], w.emb_dtype)
+            s = oracle.chunk_scores(qf, dw.emb_f(b))
+            out.append((oracle.topk(s, w.k[b]), s))
+        return out
+
+    # cycle 1: cold start (all slots empty)
+    lsa.lsa_refresh_resident(dw.dims, dw.q_emb, dw.chunk_emb, dw.K, dw.V, slots, Kr, Vr, moved, dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_OK
+    got = slots.cpu().numpy()
+    for b, (ids, s) in enumerate(oracle_ids(dw.host["q_emb"])):
+        mine = got[koff[b]:koff[b + 1]]
+        G.check_ids(np.sort(mine), ids, s, w.k[b])
+        exp, _ = oracle.refresh_resident([-1] * w.k[b], ids, w.N[b])
+        np.testing.assert_array_equal(mine, exp)
+    np.testing.assert_array_equal(moved.cpu().numpy(), w.k)
+    _check_resident(dw, got, Kr, Vr)
+
+    # cycle 2: another query; slots whose chunk stays are poisoned first and must not be rewritten
+    v = datagen.make_query_variant(w, 1)
+    q_emb2 = G.to_device(v["q_emb"], w.emb_dtype)
+    new = oracle_ids(v["q_emb"])
+    old = got.copy()
+    staying = set()
+    expected = np.empty_like(old)
+    n_copies = []
+    for b, (ids, s) in enumerate(new):
+        exp, copies = oracle.refresh_resident(old[koff[b]:koff[b + 1]], ids, w.N[b])
+        expected[koff[b]:koff[b + 1]] = exp
+        n_copies.append(len(copies))
+        kept = set(ids.tolist())
+        for j, c in enumerate(old[koff[b]:koff[b + 1]]):
+            if c in kept:
+                staying.add(int(koff[b]) + j)
+    for g in staying:
+        Kr[g * w.C:(g + 1) * w.C] = 7.0
+        Vr[g * w.C:(g + 1) * w.C] = -7.0
+    lsa.lsa_refresh_resident(dw.dims, q_emb2, dw.chunk_emb, dw.K, dw.V, slots, Kr, Vr, moved, dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_OK
+    np.testing.assert_array_equal(slots.cpu().numpy(), expected)
+    np.testing.assert_array_equal(moved.cpu().numpy(), n_copies)
+    assert sum(n_copies) < w.total_kept or not staying
+    _check_resident(dw, expected, Kr, Vr, skip=staying)
+    for g in staying:  # untouched: still the poison
+        assert float(Kr[g * w.C:(g + 1) * w.C].float().min()) == 7.0
+        assert float(Vr[g * w.C:(g + 1) * w.C].float().max()) == -7.0
+
+    # attention over the resident buffer (slot order) equals attention over the kept set
+    for g in staying:  # restore the poisoned slots from the cache first
+        b = int(np.searchsorted(koff, g, side="right") - 1)
+        tok = oracle.kept_tokens([expected[g]], w.C)
+        Kr[g * w.C:(g + 1) * w.C] = torch.from_numpy(dw.kv_f("K", b, tok)).to(Kr.dtype).cuda()
+        Vr[g * w.C:(g + 1) * w.C] = torch.from_numpy(dw.kv_f("V", b, tok)).to(Vr.dtype).cuda()
+    lsa.lsa_sparse_decode_attn(dw.dims, dw.q, Kr, Vr, None, dw.out, dw.lse, dw.ws)
+    out = dw.out.cpu().numpy()
+    for b, (ids, _) in enumerate(new):
+        ref_o, _ = G.oracle_attention(dw, b, ids)
+        np.testing.assert_allclose(out[b], ref_o, rtol=0, atol=1e-4)

@@ -254,3 +254,36 @@ def test_planted_chunks_recovered_tiny():
     planted = datagen.planted_positions(w, 0)
     assert len(planted) == 4
     assert set(planted.tolist()) <= set(ids.tolist())
+
+
+# ---------------------------------------------------------------- resident refresh
+def test_refresh_golden():
+    g = load("refresh_slots.txt")
+    slots, copies = oracle.refresh_resident(g["old"].astype(int), g["new"].astype(int), 12)
+    np.testing.assert_array_equal(slots, g["slots"].astype(np.int32))
+    assert copies == [tuple(int(x) for x in r) for r in g["copies"]]
+
+
+def test_refresh_properties():
+    rng = np.random.default_rng(12)
+    for _ in range(200):
+        n = int(rng.integers(1, 40))
+        k = int(rng.integers(1, n + 1))
+        old = rng.permutation(n)[:k].astype(int)
+        old[rng.random(k) < 0.2] = -1                 # some empty slots
+        new = np.sort(rng.permutation(n)[:k])
+        slots, copies = oracle.refresh_resident(old, new, n)
+        assert sorted(slots.tolist()) == new.tolist()          # exactly the kept set
+        for j, c in enumerate(old):                            # kept chunks never move
+            if c in set(new.tolist()):
+                assert slots[j] == c
+        moved = {c for c, _ in copies}
+        assert moved == set(new.tolist()) - set(old.tolist())  # only entering chunks are copied
+        assert [c for c, _ in copies] == sorted(moved)         # ascending chunks ...
+        assert [j for _, j in copies] == sorted(j for _, j in copies)  # ... into ascending slots
+    # cold start: every slot empty -> the slots list the kept chunks in ascending order
+    s, c = oracle.refresh_resident([-1] * 4, [9, 3, 5, 0], 10)
+    assert s.tolist() == [0, 3, 5, 9] and len(c) == 4
+    # duplicates in a corrupt table: the chunk stays in its first slot only
+    s, _ = oracle.refresh_resident([3, 3, -1], [1, 3, 7], 8)
+    assert s.tolist() == [3, 1, 7]
