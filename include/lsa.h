@@ -116,6 +116,18 @@ LSA_API lsa_status lsa_score_chunks(const lsa_dims *dims, const void *q_emb, con
 LSA_API lsa_status lsa_topk_select(const lsa_dims *dims, const float *scores, int32_t *chunk_ids,
                            void *ws, size_t ws_bytes, void *stream);
 
+/* Threshold keep mask with a fallback floor [R3-2.3 step 5: "top-k or threshold";
+ * review section 4-3: precise-needle tasks need a threshold fallback]. The pages give no
+ * rule; this library's: k_eff = clamp(#{i : s_i >= tau}, min(k_min, k_b), k_b) and the kept
+ * set is the top-k_eff by (score desc, index asc), so the fallback keeps at least k_min chunks
+ * and the capacity k_b (dims k / k_per_seq) caps the count.
+ *   scores     [sum N_b] float32;  tau finite; k_min >= 1
+ *   chunk_ids  [sum k_b] int32, out: per sequence the k_eff kept ids ascending, then -1
+ *   kept_count [B] int32 device, out: k_eff per sequence. */
+LSA_API lsa_status lsa_threshold_select(const lsa_dims *dims, const float *scores, float tau, int32_t k_min,
+                                        int32_t *chunk_ids, int32_t *kept_count, void *ws, size_t ws_bytes,
+                                        void *stream);
+
 /* Gather of the kept chunks into a compact resident buffer [R3-2.3 step 6, ABS].
  *   K, V         [sum L_b][H][Dh]   kv_dtype (L_b = N_b * C)
  *   chunk_ids    [sum k_b]          int32, local chunk indices
@@ -187,6 +199,15 @@ LSA_API lsa_status lsa_refresh_resident(const lsa_dims *dims, const void *q_emb,
 LSA_API lsa_status lsa_sparse_decode_attn_noalloc(const lsa_dims *dims, const void *q, const void *K,
                                                   const void *V, const int32_t *chunk_ids, float *out,
                                                   float *lse, void *stream);
+
+/* The fused step with the threshold keep mask: score -> threshold select (as
+ * lsa_threshold_select) -> attention over each sequence's k_eff kept chunks (read through
+ * the ids; positions past kept_count are skipped on the device, so the host never waits).
+ * Outputs as lsa_decode_step plus kept_count_out [B] int32 device. */
+LSA_API lsa_status lsa_decode_step_threshold(const lsa_dims *dims, const void *q_emb, const void *chunk_emb,
+                                             const void *q, const void *K, const void *V, float tau,
+                                             int32_t k_min, int32_t *chunk_ids_out, int32_t *kept_count_out,
+                                             float *out, float *lse, void *ws, size_t ws_bytes, void *stream);
 
 /* Synchronise `stream`, read the sticky device error word of `ws`, clear it, and
  * return LSA_OK or the first device error (NONFINITE, BAD_ID, TIMEOUT, in that order). */

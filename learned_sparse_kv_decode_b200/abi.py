@@ -60,6 +60,9 @@ def _load():
         "lsa_get_device_status": ([vp, vp], ctypes.c_int),
         "lsa_sparse_decode_attn_noalloc": ([dp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsa_refresh_resident": ([dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+        "lsa_threshold_select": ([dp, vp, ctypes.c_float, ctypes.c_int32, vp, vp, vp, sz, vp], ctypes.c_int),
+        "lsa_decode_step_threshold": ([dp, vp, vp, vp, vp, vp, ctypes.c_float, ctypes.c_int32, vp, vp, vp, vp,
+                                       vp, sz, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -168,6 +171,18 @@ def lsa_sparse_decode_attn(dims, q, K, V, chunk_ids, out, lse, ws, stream=None) 
 def lsa_decode_step(dims, q_emb, chunk_emb, q, K, V, chunk_ids_out, out, lse, ws, stream=None) -> None:
     _check(lib.lsa_decode_step(dims.ptr, _p(q_emb), _p(chunk_emb), _p(q), _p(K), _p(V), _p(chunk_ids_out),
                                _p(out), _p(lse), _p(ws), _nbytes(ws), _stream(stream)), "lsa_decode_step")
+
+
+def lsa_threshold_select(dims, scores, tau, k_min, chunk_ids, kept_count, ws, stream=None) -> None:
+    _check(lib.lsa_threshold_select(dims.ptr, _p(scores), float(tau), int(k_min), _p(chunk_ids), _p(kept_count),
+                                    _p(ws), _nbytes(ws), _stream(stream)), "lsa_threshold_select")
+
+
+def lsa_decode_step_threshold(dims, q_emb, chunk_emb, q, K, V, tau, k_min, chunk_ids_out, kept_count_out, out,
+                              lse, ws, stream=None) -> None:
+    _check(lib.lsa_decode_step_threshold(dims.ptr, _p(q_emb), _p(chunk_emb), _p(q), _p(K), _p(V), float(tau),
+                                         int(k_min), _p(chunk_ids_out), _p(kept_count_out), _p(out), _p(lse),
+                                         _p(ws), _nbytes(ws), _stream(stream)), "lsa_decode_step_threshold")
 
 
 def lsa_refresh_resident(dims, q_emb, chunk_emb, K, V, slot_ids, K_res, V_res, moved, ws, stream=None) -> None:

@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
              const uint8_t* __restrict__ V, const int32_t* __restrict__ ids,
              float* __restrict__ part_o, float* __restrict__ part_ml, const SeqTable tab,
-             const AttnParams ap, uint32_t* err) {
+             const AttnParams ap, uint32_t* err, const int32_t* __restrict__ counts) {
     constexpr int ES = BF16 ? 2 : 4;
     constexpr int VEC = 16 / ES;   // head-dim elements per lane
     constexpr int LPH = kDh / VEC; // lanes per head
@@ -118,6 +118,7 @@ k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
     uint64_t* bars = reinterpret_cast<uint64_t*>(scratch + (kAttnConsumers / LPH) * (kDh + 2));
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kStages);
     __shared__ int s_abort;  // set by a consumer whose bounded wait gave up
+    __shared__ int s_skip[kStages];  // ring slot holds no tokens (kept position >= the sequence's count)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x, hs = blockIdx.y;
@@ -148,6 +149,12 @@ k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
                 const int64_t gidx = s / ap.SPC;
                 const int64_t within = (s % ap.SPC) * ap.TOK;
                 while (gidx >= tab.kept_off[b + 1]) ++b;
+                if (counts != nullptr && gidx - tab.kept_off[b] >= (int64_t)counts[b]) {
+                    s_skip[slot] = 1;                    // beyond this sequence's kept count
+                    mbar_arrive(full0 + 8 * slot);       // release the slot without data
+                    continue;
+                }
+                s_skip[slot] = 0;
                 int64_t token0;
                 if (ap.indexed) {
                     const int32_t id = ids[gidx];
@@ -216,7 +223,7 @@ k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
                 s_abort = 1;
                 break;
             }
-            if (active) {
+            if (active && !*(volatile int*)&s_skip[slot]) {
                 const uint32_t kb = lane_k + slot * kStageBytes;
                 const uint32_t vb = lane_v + slot * kStageBytes;
                 float sc[TPG];
@@ -296,7 +303,7 @@ k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
                 for (int e = 0; e < VEC; ++e) A[e] = 0.f;
                 for (int g = 0; g < ap.TG; ++g) {
                     const float* o = scratch + (size_t)(g * ap.HS + hl) * (kDh + 2);
-                    const float f = ex2(o[kDh] - M);
+                    const float f = M == -INFINITY ? 0.f : ex2(o[kDh] - M);  // a group may hold no tokens
                     L = fmaf(o[kDh + 1], f, L);
 #pragma unroll
                     for (int e = 0; e < VEC; ++e) A[e] = fmaf(o[li * VEC + e], f, A[e]);
@@ -426,13 +433,13 @@ cudaError_t set_split_attrs(size_t smem) {
 template <bool BF16>
 cudaError_t launch_split(cudaLaunchConfig_t* cfg, int tpg, const void* q, const void* K, const void* V,
                          const int32_t* ids, float* part_o, float* part_ml, const SeqTable& tab,
-                         const AttnParams& ap, uint32_t* err) {
+                         const AttnParams& ap, uint32_t* err, const int32_t* counts) {
     const uint8_t *q8 = (const uint8_t*)q, *K8 = (const uint8_t*)K, *V8 = (const uint8_t*)V;
     switch (tpg) {
-        case 1: return cudaLaunchKernelEx(cfg, k_attn_split<BF16, 1>, q8, K8, V8, ids, part_o, part_ml, tab, ap, err);
-        case 2: return cudaLaunchKernelEx(cfg, k_attn_split<BF16, (kTpgMax >= 2 ? 2 : 1)>, q8, K8, V8, ids, part_o, part_ml, tab, ap, err);
-        case 4: return cudaLaunchKernelEx(cfg, k_attn_split<BF16, (kTpgMax >= 4 ? 4 : 1)>, q8, K8, V8, ids, part_o, part_ml, tab, ap, err);
-        case 8: return cudaLaunchKernelEx(cfg, k_attn_split<BF16, (kTpgMax >= 8 ? 8 : 1)>, q8, K8, V8, ids, part_o, part_ml, tab, ap, err);
+        case 1: return cudaLaunchKernelEx(cfg, k_attn_split<BF16, 1>, q8, K8, V8, ids, part_o, part_ml, tab, ap, err, counts);
+        case 2: return cudaLaunchKernelEx(cfg, k_attn_split<BF16, (kTpgMax >= 2 ? 2 : 1)>, q8, K8, V8, ids, part_o, part_ml, tab, ap, err, counts);
+        case 4: return cudaLaunchKernelEx(cfg, k_attn_split<BF16, (kTpgMax >= 4 ? 4 : 1)>, q8, K8, V8, ids, part_o, part_ml, tab, ap, err, counts);
+        case 8: return cudaLaunchKernelEx(cfg, k_attn_split<BF16, (kTpgMax >= 8 ? 8 : 1)>, q8, K8, V8, ids, part_o, part_ml, tab, ap, err, counts);
     }
     return cudaErrorInvalidValue;
 }
@@ -491,7 +498,7 @@ cudaError_t attn_ctas_per_device(lsa_dtype kv, int num_sms, int* out) {
 cudaError_t launch_attention(const lsa_dims& d, const SeqTable& tab, int ctas_per_device,
                              const void* q, const void* K, const void* V, const int32_t* ids,
                              float* part_o, float* part_ml, float* out, float* lse, uint32_t* err,
-                             cudaStream_t stream, bool pdl) {
+                             cudaStream_t stream, bool pdl, const int32_t* counts) {
     const AttnLaunch L = plan_attention(d, tab, ctas_per_device, ids != nullptr);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -507,8 +514,8 @@ cudaError_t launch_attention(const lsa_dims& d, const SeqTable& tab, int ctas_pe
     if (L.tpg != 1 && L.tpg != 2 && L.tpg != 4 && L.tpg != 8) return cudaErrorInvalidValue;
     if ((int64_t)L.ap.G > kMergeMaxSlots) return cudaErrorInvalidValue;
     cudaError_t e = d.kv_dtype == LSA_BF16
-                        ? launch_split<true>(&cfg, L.tpg, q, K, V, ids, part_o, part_ml, tab, L.ap, err)
-                        : launch_split<false>(&cfg, L.tpg, q, K, V, ids, part_o, part_ml, tab, L.ap, err);
+                        ? launch_split<true>(&cfg, L.tpg, q, K, V, ids, part_o, part_ml, tab, L.ap, err, counts)
+                        : launch_split<false>(&cfg, L.tpg, q, K, V, ids, part_o, part_ml, tab, L.ap, err, counts);
     if (e != cudaSuccess) return e;
 
     cudaLaunchConfig_t mcfg = {};

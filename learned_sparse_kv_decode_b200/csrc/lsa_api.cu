@@ -15,6 +15,9 @@ cudaError_t launch_score(const lsa_dims& d, const SeqTable& tab, int max_n, cons
 bool score_uses_umma(const lsa_dims& d);
 cudaError_t launch_topk(const lsa_dims& d, const SeqTable& tab, int max_n, const float* scores,
                         int32_t* ids, uint32_t* err, cudaStream_t stream, bool pdl);
+cudaError_t launch_threshold(const lsa_dims& d, const SeqTable& tab, int max_n, const float* scores,
+                             float tau, int k_min, int32_t* ids, int32_t* counts, uint32_t* err,
+                             cudaStream_t stream, bool pdl);
 cudaError_t launch_gather(const lsa_dims& d, const SeqTable& tab, const void* K, const void* V,
                           const int32_t* ids, void* K_res, void* V_res, uint32_t* err,
                           cudaStream_t stream);
@@ -30,7 +33,7 @@ cudaError_t launch_refresh(const lsa_dims& d, const SeqTable& tab, int max_n, co
 cudaError_t launch_attention(const lsa_dims& d, const SeqTable& tab, int ctas_per_device,
                              const void* q, const void* K, const void* V, const int32_t* ids,
                              float* part_o, float* part_ml, float* out, float* lse, uint32_t* err,
-                             cudaStream_t stream, bool pdl);
+                             cudaStream_t stream, bool pdl, const int32_t* counts = nullptr);
 }  // namespace lsa
 
 using namespace lsa;
@@ -280,6 +283,48 @@ lsa_status lsa_decode_step(const lsa_dims* dims, const void* q_emb, const void* 
     e = launch_attention(*dims, p.tab, di.attn_ctas[dims->kv_dtype], q, K, V, chunk_ids_out,
                          reinterpret_cast<float*>(at(ws, w.part_o)),
                          reinterpret_cast<float*>(at(ws, w.part_ml)), out, lse, err, st, true);
+    return cuda_status(e);
+}
+
+lsa_status lsa_threshold_select(const lsa_dims* dims, const float* scores, float tau, int32_t k_min,
+                                int32_t* chunk_ids, int32_t* kept_count, void* ws, size_t ws_bytes,
+                                void* stream) {
+    Prepared p;
+    DeviceInfo di;
+    WsLayout w;
+    lsa_status s = prepare_ws(dims, ws, ws_bytes, &p, &di, &w);
+    if (s != LSA_OK) return s;
+    if (!aligned16(scores) || !aligned16(chunk_ids) || !aligned16(kept_count)) return LSA_ERR_INVALID_ARG;
+    if (k_min < 1 || !std::isfinite(tau)) return LSA_ERR_INVALID_ARG;
+    return cuda_status(launch_threshold(*dims, p.tab, p.max_n, scores, tau, k_min, chunk_ids, kept_count,
+                                        reinterpret_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream),
+                                        false));
+}
+
+lsa_status lsa_decode_step_threshold(const lsa_dims* dims, const void* q_emb, const void* chunk_emb,
+                                     const void* q, const void* K, const void* V, float tau, int32_t k_min,
+                                     int32_t* chunk_ids_out, int32_t* kept_count_out, float* out, float* lse,
+                                     void* ws, size_t ws_bytes, void* stream) {
+    Prepared p;
+    DeviceInfo di;
+    WsLayout w;
+    lsa_status s = prepare_ws(dims, ws, ws_bytes, &p, &di, &w);
+    if (s != LSA_OK) return s;
+    if (!aligned16(q_emb) || !aligned16(chunk_emb) || !aligned16(q) || !aligned16(K) || !aligned16(V) ||
+        !aligned16(chunk_ids_out) || !aligned16(kept_count_out) || !aligned16(out))
+        return LSA_ERR_INVALID_ARG;
+    if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LSA_ERR_INVALID_ARG;
+    if (k_min < 1 || !std::isfinite(tau)) return LSA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+    float* scores = reinterpret_cast<float*>(at(ws, w.scores));
+    cudaError_t e = launch_score(*dims, p.tab, p.max_n, q_emb, chunk_emb, scores, err, di.sms, st, false);
+    if (e == cudaSuccess)
+        e = launch_threshold(*dims, p.tab, p.max_n, scores, tau, k_min, chunk_ids_out, kept_count_out, err, st, true);
+    if (e == cudaSuccess)
+        e = launch_attention(*dims, p.tab, di.attn_ctas[dims->kv_dtype], q, K, V, chunk_ids_out,
+                             reinterpret_cast<float*>(at(ws, w.part_o)),
+                             reinterpret_cast<float*>(at(ws, w.part_ml)), out, lse, err, st, true, kept_count_out);
     return cuda_status(e);
 }
 

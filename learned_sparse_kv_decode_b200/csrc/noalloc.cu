@@ -32,7 +32,7 @@ cudaError_t attn_ctas_per_device(lsa_dtype kv, int num_sms, int* out);
 cudaError_t launch_attention(const lsa_dims& d, const SeqTable& tab, int ctas_per_device,
                              const void* q, const void* K, const void* V, const int32_t* ids,
                              float* part_o, float* part_ml, float* out, float* lse, uint32_t* err,
-                             cudaStream_t stream, bool pdl);
+                             cudaStream_t stream, bool pdl, const int32_t* counts = nullptr);
 }  // namespace lsa
 
 using namespace lsa;

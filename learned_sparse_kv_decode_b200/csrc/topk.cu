@@ -60,12 +60,50 @@ __device__ __forceinline__ uint32_t dsmem_ld(const uint32_t* p, uint32_t rank) {
     return v;
 }
 
+// Threshold keep mask (review section 3-2 (3), step 5: "top-k or threshold"): keep the
+// chunks scoring at least tau, but no fewer than k_min (the fallback floor) and no more than
+// the capacity k_b, always as a top-k set: k_eff = clamp(#{s >= tau}, min(k_min, k_b), k_b).
+// counts[b] receives k_eff; id positions k_eff .. k_b-1 are set to -1.
+struct ThresholdArgs {
+    int enabled;
+    float tau;
+    int k_min;
+    int32_t* counts;
+};
+
+// Sum of one value per thread over the CTA and then the cluster (every thread gets the total).
+// `red` holds one slot per warp, `cta_total` one word that the cluster reads through DSMEM.
+template <int WARPS>
+__device__ __forceinline__ uint32_t cluster_sum(uint32_t v, uint32_t* red, uint32_t* cta_total, uint32_t cs) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    v = __reduce_add_sync(0xffffffffu, v);
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    uint32_t t = 0;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) t += red[w];
+    if (cs == 1) {
+        __syncthreads();  // red is reused by the caller
+        return t;
+    }
+    if (threadIdx.x == 0) *cta_total = t;
+    cluster_sync_all();
+    uint32_t parts[kTopkMaxCluster];
+#pragma unroll
+    for (int r = 0; r < kTopkMaxCluster; ++r) parts[r] = (uint32_t)r < cs ? dsmem_ld(cta_total, r) : 0u;
+    uint32_t sum = 0;
+#pragma unroll
+    for (int r = 0; r < kTopkMaxCluster; ++r) sum += parts[r];
+    cluster_sync_all();  // every CTA has read cta_total and red before they are reused
+    return sum;
+}
+
 // grid (CS, B) with cluster (CS, 1, 1), 1024 threads.
 // SMEM_KEYS: the CTA's key slice is cached in dynamic shared memory.
 template <bool SMEM_KEYS>
 __global__ void __launch_bounds__(kTopkThreads)
 k_topk(const float* __restrict__ scores, int32_t* __restrict__ ids, const SeqTable tab,
-       uint32_t* err) {
+       uint32_t* err, const ThresholdArgs th) {
     extern __shared__ uint32_t skeys[];
     __shared__ uint32_t hist[2][256];  // double-buffered: pass p uses hist[p & 1]
     __shared__ uint32_t tot[256];
@@ -74,12 +112,14 @@ k_topk(const float* __restrict__ scores, int32_t* __restrict__ ids, const SeqTab
     __shared__ uint32_t o_gt[kTopkWarps], o_eq[kTopkWarps];
     __shared__ uint32_t t_gt, t_eq;
     __shared__ uint32_t c_gt, c_eq;  // this CTA's totals of keys > T and == T (read by the cluster)
+    __shared__ uint32_t s_red[kTopkWarps], s_cnt;
 
     const int b = blockIdx.y;
     const uint32_t rank = cluster_rank(), cs = cluster_size();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n = tab.chunk_off[b + 1] - tab.chunk_off[b];
-    const int k = tab.kept_off[b + 1] - tab.kept_off[b];
+    const int kcap = tab.kept_off[b + 1] - tab.kept_off[b];
+    int k = kcap;
     const int slice = (n + (int)cs - 1) / (int)cs;
     const int lo = min(n, (int)rank * slice), hi = min(n, lo + slice);
     const int m = hi - lo;  // keys owned by this CTA: indices [lo, hi)
@@ -106,6 +146,14 @@ k_topk(const float* __restrict__ scores, int32_t* __restrict__ ids, const SeqTab
         }
     };
 
+    if (th.enabled) {
+        bool dummy = false;
+        const uint32_t tkey = score_key(th.tau, dummy);
+        uint32_t c = 0;
+        for (int i = tid; i < m; i += kTopkThreads) c += key_at(i) >= tkey;
+        const int total = (int)cluster_sum<kTopkWarps>(c, s_red, &s_cnt, cs);
+        k = max(min(total, kcap), min(th.k_min, kcap));
+    }
     uint32_t prefix = 0, need = (uint32_t)k;
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
@@ -263,6 +311,10 @@ k_topk(const float* __restrict__ scores, int32_t* __restrict__ ids, const SeqTab
         carry_eq += t_eq;
         __syncthreads();
     }
+    if (th.enabled) {
+        for (int pos = k + (int)rank * kTopkThreads + tid; pos < kcap; pos += (int)cs * kTopkThreads) out[pos] = -1;
+        if (rank == 0 && tid == 0) th.counts[b] = k;
+    }
     if (cs > 1) cluster_sync_all();  // keep this CTA's shared memory alive until the cluster is done reading it
 }
 
@@ -317,17 +369,19 @@ __device__ __forceinline__ void find_digit(const uint32_t* h256, uint32_t need, 
 template <int R>
 __global__ void __launch_bounds__(kTopkRegThreads)
 k_topk_reg(const float* __restrict__ scores, int32_t* __restrict__ ids, const SeqTable tab,
-           uint32_t* err) {
+           uint32_t* err, const ThresholdArgs th) {
     __shared__ uint32_t hist[3][256];
     __shared__ uint32_t tot[256];
     __shared__ uint32_t w_gt[kTopkRegWarps], w_eq[kTopkRegWarps];
     __shared__ uint32_t c_gt, c_eq;  // this CTA's totals of keys > T and == T (read by the cluster)
+    __shared__ uint32_t s_red[kTopkRegWarps], s_cnt;
 
     const int b = blockIdx.y;
     const uint32_t rank = cluster_rank(), cs = cluster_size();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n = tab.chunk_off[b + 1] - tab.chunk_off[b];
-    const int k = tab.kept_off[b + 1] - tab.kept_off[b];
+    const int kcap = tab.kept_off[b + 1] - tab.kept_off[b];
+    int k = kcap;
     const int slice = (n + (int)cs - 1) / (int)cs;
     const int lo = min(n, (int)rank * slice), hi = min(n, lo + slice);
     const int m = hi - lo;                     // keys of this CTA: [lo, hi)
@@ -349,6 +403,15 @@ k_topk_reg(const float* __restrict__ scores, int32_t* __restrict__ ids, const Se
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(err, kErrNonFinite);
     __syncthreads();
 
+    if (th.enabled) {
+        bool dummy = false;
+        const uint32_t tkey = score_key(th.tau, dummy);
+        uint32_t c = 0;
+#pragma unroll
+        for (int j = 0; j < R; ++j) c += (base + j < m && kr[j] >= tkey) ? 1u : 0u;
+        const int total = (int)cluster_sum<kTopkRegWarps>(c, s_red, &s_cnt, cs);
+        k = max(min(total, kcap), min(th.k_min, kcap));
+    }
     uint32_t prefix = 0, need = (uint32_t)k;
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
@@ -459,6 +522,11 @@ k_topk_reg(const float* __restrict__ scores, int32_t* __restrict__ ids, const Se
             }
         }
     }
+    if (th.enabled) {
+        for (int pos = k + (int)rank * kTopkRegThreads + tid; pos < kcap; pos += (int)cs * kTopkRegThreads)
+            out[pos] = -1;
+        if (rank == 0 && tid == 0) th.counts[b] = k;
+    }
     if (cs > 1) cluster_sync_all();  // keep c_gt / c_eq alive until every CTA has read them
 }
 
@@ -480,8 +548,8 @@ int topk_cluster_size(int max_n) {
     return cs;
 }
 
-cudaError_t launch_topk(const lsa_dims& d, const SeqTable& tab, int max_n, const float* scores,
-                        int32_t* ids, uint32_t* err, cudaStream_t stream, bool pdl) {
+cudaError_t launch_topk_impl(const lsa_dims& d, const SeqTable& tab, int max_n, const float* scores,
+                             int32_t* ids, uint32_t* err, cudaStream_t stream, bool pdl, const ThresholdArgs& th) {
     const int cs = topk_cluster_size(max_n);
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
@@ -500,20 +568,33 @@ cudaError_t launch_topk(const lsa_dims& d, const SeqTable& tab, int max_n, const
     if (per_thread <= 16) {
         cfg.blockDim = dim3(kTopkRegThreads, 1, 1);
         cfg.dynamicSmemBytes = 0;
-        if (per_thread <= 1) return cudaLaunchKernelEx(&cfg, k_topk_reg<1>, scores, ids, tab, err);
-        if (per_thread <= 2) return cudaLaunchKernelEx(&cfg, k_topk_reg<2>, scores, ids, tab, err);
-        if (per_thread <= 4) return cudaLaunchKernelEx(&cfg, k_topk_reg<4>, scores, ids, tab, err);
-        if (per_thread <= 8) return cudaLaunchKernelEx(&cfg, k_topk_reg<8>, scores, ids, tab, err);
-        return cudaLaunchKernelEx(&cfg, k_topk_reg<16>, scores, ids, tab, err);
+        if (per_thread <= 1) return cudaLaunchKernelEx(&cfg, k_topk_reg<1>, scores, ids, tab, err, th);
+        if (per_thread <= 2) return cudaLaunchKernelEx(&cfg, k_topk_reg<2>, scores, ids, tab, err, th);
+        if (per_thread <= 4) return cudaLaunchKernelEx(&cfg, k_topk_reg<4>, scores, ids, tab, err, th);
+        if (per_thread <= 8) return cudaLaunchKernelEx(&cfg, k_topk_reg<8>, scores, ids, tab, err, th);
+        return cudaLaunchKernelEx(&cfg, k_topk_reg<16>, scores, ids, tab, err, th);
     }
     cfg.blockDim = dim3(kTopkThreads, 1, 1);
     const size_t key_bytes = (size_t)slice * 4;
     if (key_bytes <= kTopkSmemKeyLimit) {
         cfg.dynamicSmemBytes = key_bytes;
-        return cudaLaunchKernelEx(&cfg, k_topk<true>, scores, ids, tab, err);
+        return cudaLaunchKernelEx(&cfg, k_topk<true>, scores, ids, tab, err, th);
     }
     cfg.dynamicSmemBytes = 0;
-    return cudaLaunchKernelEx(&cfg, k_topk<false>, scores, ids, tab, err);
+    return cudaLaunchKernelEx(&cfg, k_topk<false>, scores, ids, tab, err, th);
+}
+
+cudaError_t launch_topk(const lsa_dims& d, const SeqTable& tab, int max_n, const float* scores,
+                        int32_t* ids, uint32_t* err, cudaStream_t stream, bool pdl) {
+    const ThresholdArgs none = {0, 0.f, 0, nullptr};
+    return launch_topk_impl(d, tab, max_n, scores, ids, err, stream, pdl, none);
+}
+
+cudaError_t launch_threshold(const lsa_dims& d, const SeqTable& tab, int max_n, const float* scores,
+                             float tau, int k_min, int32_t* ids, int32_t* counts, uint32_t* err,
+                             cudaStream_t stream, bool pdl) {
+    const ThresholdArgs th = {1, tau, k_min, counts};
+    return launch_topk_impl(d, tab, max_n, scores, ids, err, stream, pdl, th);
 }
 
 }  // namespace lsa

@@ -17,7 +17,8 @@ dimensionstp.github.io, section 3-2 (2)-(3); arXiv abstract):
    scale 1/sqrt(Dh), returning the output and the log-sum-exp per head;
 5. footprint = k * chunk_len / L;
 6. the retrieval cycle's resident refresh (review section 3-1 "retrieval interval" and
-   section 3-2 (3) step 7): the slot table after a cycle, written out as its rule.
+   section 3-2 (3) step 7): the slot table after a cycle, written out as its rule;
+7. the threshold keep mask with a fallback floor (section 3-2 (3) step 5).
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (hand-worked fixtures in ``tests/golden/``, closed forms, a brute-force
@@ -161,3 +162,14 @@ def refresh_resident(old_slots, new_ids, n: int):
         slots[j] = c
         copies.append((c, j))
     return np.array(slots, dtype=np.int32), copies
+
+
+def threshold_select(scores, tau: float, k_min: int, k_max: int) -> np.ndarray:
+    """Threshold keep mask with a fallback floor (review section 3-2 (3) step 5, "top-k or
+    threshold"; section 4-3: precise-needle tasks need a threshold fallback). The pages give
+    no rule; the one taken: k_eff = clamp(#{s >= tau}, min(k_min, k_max), k_max), and the kept
+    set is the top-k_eff (score desc, index asc), reported ascending."""
+    s = _f64(scores)
+    count = int(np.count_nonzero(s >= float(tau)))
+    k_eff = min(max(count, min(int(k_min), int(k_max))), int(k_max))
+    return topk(s, k_eff)

@@ -417,3 +417,55 @@ def test_refresh_resident_cycles(lsa, case):
     for b, (ids, _) in enumerate(new):
         ref_o, _ = G.oracle_attention(dw, b, ids)
         np.testing.assert_allclose(out[b], ref_o, rtol=0, atol=1e-4)
+
+
+# ------------------------------------------------------------------ threshold keep mask
+@pytest.mark.parametrize("N,kmax", [((64,), (64,)), ((7, 2048), (7, 300)), ((5000, 16384), (900, 2500)),
+                                    ((60000,), (9000,))])
+@pytest.mark.parametrize("tau_kind", ["cap", "mid", "floor", "tie"])
+def test_threshold_select_bit_exact(lsa, N, kmax, tau_kind):
+    w = datagen.small_workload(B=len(N), N=N, k=kmax, E=64)
+    dims = G.dims_of(w, lsa)
+    ws = lsa.alloc_workspace(dims)
+    s = np.concatenate([_tie_scores(n, 300 + i) for i, n in enumerate(N)])
+    tau = {"cap": -100.0, "mid": 0.75, "floor": 100.0, "tie": float(s[3])}[tau_kind]
+    k_min = 3
+    ids = torch.full((w.total_kept,), 12345, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(w.B, dtype=torch.int32, device="cuda")
+    lsa.lsa_threshold_select(dims, torch.from_numpy(s).cuda(), np.float32(tau), k_min, ids, cnt, ws)
+    assert lsa.lsa_get_device_status(ws) == lsa.LSA_OK
+    got, got_cnt = ids.cpu().numpy(), cnt.cpu().numpy()
+    off, koff = w.chunk_offsets, w.k_offsets
+    for b in range(w.B):
+        ref = oracle.threshold_select(s[off[b]:off[b + 1]].astype(np.float64), np.float32(tau), k_min, kmax[b])
+        assert got_cnt[b] == len(ref)
+        np.testing.assert_array_equal(got[koff[b]:koff[b] + len(ref)], ref)
+        assert (got[koff[b] + len(ref):koff[b + 1]] == -1).all()
+
+
+@pytest.mark.parametrize("case", STEP_CASES[:4], ids=lambda c: f"B{c['B']}-E{c['E']}-Q{c.get('Q', 1)}-H{c['H']}")
+def test_decode_step_threshold(lsa, case):
+    w = datagen.small_workload(seed=66, **dict(case))
+    dw = G.DeviceWorkload(w, lsa)
+    # tau between the scores: about a third of each sequence's chunks pass (capacity k_b)
+    all_s = [oracle.chunk_scores(dw.q_emb_f(b), dw.emb_f(b)) for b in range(w.B)]
+    tau = np.float32(np.median(np.concatenate(all_s)) + 0.5 * np.std(np.concatenate(all_s)))
+    k_min = 1
+    cnt = torch.zeros(w.B, dtype=torch.int32, device="cuda")
+    lsa.lsa_decode_step_threshold(dw.dims, dw.q_emb, dw.chunk_emb, dw.q, dw.K, dw.V, tau, k_min, dw.ids, cnt,
+                                  dw.out, dw.lse, dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_OK
+    got, got_cnt, out = dw.ids.cpu().numpy(), cnt.cpu().numpy(), dw.out.cpu().numpy()
+    koff = w.k_offsets
+    for b in range(w.B):
+        s = all_s[b]
+        ref = oracle.threshold_select(s, tau, k_min, w.k[b])
+        near = np.abs(s - float(tau)) <= G.NEAR_TIE_RTOL * max(abs(float(tau)), 1.0)
+        if not near.any():
+            assert got_cnt[b] == len(ref)
+        k_eff = int(got_cnt[b])
+        mine = got[koff[b]:koff[b] + k_eff]
+        if k_eff == len(ref):
+            G.check_ids(mine, ref, s, k_eff)
+        ref_o, _ = G.oracle_attention(dw, b, mine)
+        np.testing.assert_allclose(out[b], ref_o, rtol=0, atol=1e-4)

@@ -287,3 +287,31 @@ def test_refresh_properties():
     # duplicates in a corrupt table: the chunk stays in its first slot only
     s, _ = oracle.refresh_resident([3, 3, -1], [1, 3, 7], 8)
     assert s.tolist() == [3, 1, 7]
+
+
+# ---------------------------------------------------------------- threshold keep mask
+@pytest.mark.parametrize("case", [1, 2, 3, 4, 5])
+def test_threshold_golden(case):
+    g = load("threshold_select.txt")
+    ids = oracle.threshold_select(g["scores"], g[f"tau{case}"], int(g[f"kmin{case}"]), int(g[f"kmax{case}"]))
+    np.testing.assert_array_equal(ids, np.atleast_1d(g[f"ids{case}"]).astype(np.int32))
+
+
+def test_threshold_properties():
+    rng = np.random.default_rng(13)
+    for _ in range(200):
+        n = int(rng.integers(1, 60))
+        s = np.round(rng.standard_normal(n) * 3) / 2  # ties
+        tau = float(rng.choice(s)) if rng.random() < 0.5 else float(rng.standard_normal())
+        k_max = int(rng.integers(1, n + 1))
+        k_min = int(rng.integers(1, k_max + 1))
+        ids = oracle.threshold_select(s, tau, k_min, k_max)
+        passing = np.flatnonzero(s >= tau)
+        assert k_min <= len(ids) <= k_max
+        if k_min <= len(passing) <= k_max:       # the threshold alone decides
+            np.testing.assert_array_equal(ids, passing)
+        elif len(passing) < k_min:              # fallback: every passing chunk is kept, plus the best others
+            assert set(passing.tolist()) <= set(ids.tolist())
+        else:                                    # cap: all kept chunks pass
+            assert (s[ids] >= tau).all()
+        np.testing.assert_array_equal(ids, oracle.topk(s, len(ids)))  # always a top-k set
