@@ -336,3 +336,58 @@ def make_query_variant(w: Workload, r: int) -> dict:
     q_emb = normal_f32(seed, TENSOR_IDS["q_emb"], np.arange(w.B * w.Q * w.E)).reshape(w.B, w.Q, w.E)
     q = normal_f32(seed, TENSOR_IDS["q"], np.arange(w.B * w.H * w.Dh)).reshape(w.B, w.H, w.Dh)
     return {"q_emb": _store(q_emb, w.emb_dtype), "q": _store(q, w.kv_dtype)}
+
+
+TENSOR_IDS.update({"idx_q": 11, "idx_k": 12, "idx_qs": 13, "idx_ks": 14, "idx_w": 15, "idx_plant": 16})
+
+
+def e4m3_bits(x: np.ndarray) -> np.ndarray:
+    """float32 -> float8_e4m3 bit patterns (round to nearest even, saturated to +-448)."""
+    import torch
+    t = torch.from_numpy(np.clip(np.asarray(x, dtype=np.float32), -448.0, 448.0))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy().copy()
+
+
+def make_indexer_inputs(w: Workload, layers: int = 3, heads: int = 128, dim: int = 128) -> dict:
+    """Inputs of the FP8 compressed-K indexer score for a workload.
+
+    compressed_k [layers][sum N][132] uint8 (128 e4m3 key values + float32 scale), q_fp8
+    [B][layers][heads][dim] e4m3, q_scale [B][layers][heads] and head_w [layers][heads]
+    float32. Keys and queries are N(0, 8^2) before quantisation, both dequant scales are
+    about 1/27 (so a dequantised head logit is about N(0, 1)) and the head weights are
+    N(0, 1) / (4 sqrt(heads)). In every layer, the chunks of `planted_positions` copy (plus
+    0.5 noise) the query of that layer's head with the largest weight, so they score high."""
+    n = w.total_chunks
+    q = normal_f32(w.seed, TENSOR_IDS["idx_q"], np.arange(w.B * layers * heads * dim))
+    q = (q * np.float32(8.0)).reshape(w.B, layers, heads, dim)
+    q8 = e4m3_bits(q)
+    qv = e4m3_bits_to_f32(q8)
+    k = normal_f32(w.seed, TENSOR_IDS["idx_k"], np.arange(layers * n * dim))
+    k = (k * np.float32(8.0)).reshape(layers, n, dim)
+    hw = (normal_f32(w.seed, TENSOR_IDS["idx_w"], np.arange(layers * heads)).reshape(layers, heads)
+          / np.float32(4.0 * math.sqrt(heads))).astype(np.float32)
+    off = w.chunk_offsets
+    for b in range(w.B):
+        pos = planted_positions(w, b) if w.plant_count else np.zeros(0, np.int64)
+        for l in range(layers):
+            hstar = int(np.argmax(hw[l]))
+            noise = normal_f32(w.seed, TENSOR_IDS["idx_plant"] + (l << 8),
+                               (off[b] + pos)[:, None] * dim + np.arange(dim)[None, :])
+            k[l, off[b] + pos] = qv[b, l, hstar][None, :] + np.float32(0.5) * noise
+    k8 = e4m3_bits(k)
+    base = np.float32(1.0 / 27.0)
+    ks = base * (np.float32(1.0) + np.float32(0.1) * uniform_f64(w.seed, TENSOR_IDS["idx_ks"],
+                                                                  np.arange(layers * n)).astype(np.float32))
+    qs = base * (np.float32(1.0) + np.float32(0.1) * uniform_f64(w.seed, TENSOR_IDS["idx_qs"],
+                                                                  np.arange(w.B * layers * heads)).astype(np.float32))
+    ck = np.empty((layers, n, dim + 4), dtype=np.uint8)
+    ck[..., :dim] = k8
+    ck[..., dim:] = ks.astype("<f4").reshape(layers, n, 1).view(np.uint8).reshape(layers, n, 4)
+    return {"compressed_k": ck, "q_fp8": q8, "q_scale": qs.reshape(w.B, layers, heads).astype(np.float32),
+            "head_w": hw, "layers": layers, "heads": heads}
+
+
+def e4m3_bits_to_f32(codes: np.ndarray) -> np.ndarray:
+    """float8_e4m3 bit patterns -> float32 (input construction only)."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8)).view(torch.float8_e4m3fn).float().numpy()

@@ -54,6 +54,7 @@ extern "C" {
 #define LSA_ABI_VERSION 1
 #define LSA_MAX_BATCH 256   /* sequences per call */
 #define LSA_HEAD_DIM 128    /* Dh: the pages' HEAD_DIM (review, section 4-3) */
+#define LSA_INDEX_DIM 128   /* compressed-K key dim: 128 e4m3 values per 132-byte chunk (review, section 3-2 (1)) */
 
 typedef enum {
     LSA_OK = 0,
@@ -67,6 +68,9 @@ typedef enum {
 } lsa_status;
 
 typedef enum { LSA_F32 = 0, LSA_BF16 = 1 } lsa_dtype;
+
+/* How the per-layer indexer scores are combined (review, section 3-2 (2): max or mean). */
+typedef enum { LSA_ENSEMBLE_MAX = 0, LSA_ENSEMBLE_MEAN = 1 } lsa_ensemble;
 
 /* Problem shape of one call. Host memory; copied by value into the launch. */
 typedef struct {
@@ -106,6 +110,22 @@ LSA_API lsa_status lsa_workspace_init(void *ws, size_t ws_bytes, void *stream);
  * embeddings and E <= 256 runs a tcgen05 tensor-core GEMM with a per-row max. */
 LSA_API lsa_status lsa_score_chunks(const lsa_dims *dims, const void *q_emb, const void *chunk_emb,
                             float *scores, void *ws, size_t ws_bytes, void *stream);
+
+/* The Neural Memory Indexer's score on FP8 compressed-K chunks [R3-2.2; review sections
+ * 3-2 (1) (the 132-byte chunk format) and 4-3 (128 heads x 128 dims)]:
+ *   s_i = ensemble_l sigmoid( sum_h w_lh * ReLU( ks_li * qs_blh * (q8_blh . k8_li) ) )
+ *   compressed_k [L][sum N_b][132] bytes: 128 float8_e4m3 key values, then the float32
+ *                dequant scale ks (little-endian), per layer and chunk
+ *   q_fp8        [B][L][n_heads][128] float8_e4m3 queries (the query-side projection, norm,
+ *                RoPE and Hadamard transform happen before this call)
+ *   q_scale      [B][L][n_heads] float32 query dequant scales;  head_w [L][n_heads] float32
+ *   scores       [sum N_b] float32, out
+ * dims->E must be LSA_INDEX_DIM; n_layers 1..16; n_heads a multiple of 16 in 16..256.
+ * A tcgen05 kind::f8f6f4 tensor-core GEMM (e4m3 x e4m3 -> fp32 in TMEM) per layer. */
+LSA_API lsa_status lsa_indexer_score_fp8(const lsa_dims *dims, int32_t n_layers, int32_t n_heads,
+                                         lsa_ensemble ensemble, const void *compressed_k, const void *q_fp8,
+                                         const float *q_scale, const float *head_w, float *scores, void *ws,
+                                         size_t ws_bytes, void *stream);
 
 /* Top-k keep mask [R3-2.3 step 5].
  *   scores    [sum N_b]   float32
@@ -208,6 +228,15 @@ LSA_API lsa_status lsa_decode_step_threshold(const lsa_dims *dims, const void *q
                                              const void *q, const void *K, const void *V, float tau,
                                              int32_t k_min, int32_t *chunk_ids_out, int32_t *kept_count_out,
                                              float *out, float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/* The fused step with the FP8 indexer score: lsa_indexer_score_fp8 -> top-k -> attention
+ * over the kept chunks (as lsa_decode_step, whose q_emb/chunk_emb are replaced by the
+ * indexer inputs). */
+LSA_API lsa_status lsa_decode_step_fp8(const lsa_dims *dims, int32_t n_layers, int32_t n_heads,
+                                       lsa_ensemble ensemble, const void *compressed_k, const void *q_fp8,
+                                       const float *q_scale, const float *head_w, const void *q, const void *K,
+                                       const void *V, int32_t *chunk_ids_out, float *out, float *lse, void *ws,
+                                       size_t ws_bytes, void *stream);
 
 /* Synchronise `stream`, read the sticky device error word of `ws`, clear it, and
  * return LSA_OK or the first device error (NONFINITE, BAD_ID, TIMEOUT, in that order). */

@@ -21,6 +21,8 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "lsa.h")
 LSA_OK, LSA_ERR_INVALID_ARG, LSA_ERR_WORKSPACE, LSA_ERR_CUDA = 0, 1, 2, 3
 LSA_ERR_NONFINITE, LSA_ERR_TIMEOUT, LSA_ERR_UNSUPPORTED, LSA_ERR_BAD_ID = 4, 5, 6, 7
 LSA_F32, LSA_BF16 = 0, 1
+LSA_ENSEMBLE_MAX, LSA_ENSEMBLE_MEAN = 0, 1
+LSA_INDEX_DIM = 128
 LSA_MAX_BATCH = 256
 LSA_HEAD_DIM = 128
 
@@ -63,6 +65,10 @@ def _load():
         "lsa_threshold_select": ([dp, vp, ctypes.c_float, ctypes.c_int32, vp, vp, vp, sz, vp], ctypes.c_int),
         "lsa_decode_step_threshold": ([dp, vp, vp, vp, vp, vp, ctypes.c_float, ctypes.c_int32, vp, vp, vp, vp,
                                        vp, sz, vp], ctypes.c_int),
+        "lsa_indexer_score_fp8": ([dp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int, vp, vp, vp, vp, vp, vp, sz, vp],
+                                  ctypes.c_int),
+        "lsa_decode_step_fp8": ([dp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp,
+                                 vp, vp, vp, sz, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -171,6 +177,20 @@ def lsa_sparse_decode_attn(dims, q, K, V, chunk_ids, out, lse, ws, stream=None) 
 def lsa_decode_step(dims, q_emb, chunk_emb, q, K, V, chunk_ids_out, out, lse, ws, stream=None) -> None:
     _check(lib.lsa_decode_step(dims.ptr, _p(q_emb), _p(chunk_emb), _p(q), _p(K), _p(V), _p(chunk_ids_out),
                                _p(out), _p(lse), _p(ws), _nbytes(ws), _stream(stream)), "lsa_decode_step")
+
+
+def lsa_indexer_score_fp8(dims, n_layers, n_heads, ensemble, compressed_k, q_fp8, q_scale, head_w, scores, ws,
+                          stream=None) -> None:
+    _check(lib.lsa_indexer_score_fp8(dims.ptr, int(n_layers), int(n_heads), int(ensemble), _p(compressed_k),
+                                     _p(q_fp8), _p(q_scale), _p(head_w), _p(scores), _p(ws), _nbytes(ws),
+                                     _stream(stream)), "lsa_indexer_score_fp8")
+
+
+def lsa_decode_step_fp8(dims, n_layers, n_heads, ensemble, compressed_k, q_fp8, q_scale, head_w, q, K, V,
+                        chunk_ids_out, out, lse, ws, stream=None) -> None:
+    _check(lib.lsa_decode_step_fp8(dims.ptr, int(n_layers), int(n_heads), int(ensemble), _p(compressed_k),
+                                   _p(q_fp8), _p(q_scale), _p(head_w), _p(q), _p(K), _p(V), _p(chunk_ids_out),
+                                   _p(out), _p(lse), _p(ws), _nbytes(ws), _stream(stream)), "lsa_decode_step_fp8")
 
 
 def lsa_threshold_select(dims, scores, tau, k_min, chunk_ids, kept_count, ws, stream=None) -> None:

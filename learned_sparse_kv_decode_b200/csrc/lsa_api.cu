@@ -25,6 +25,11 @@ cudaError_t attn_ctas_per_device(lsa_dtype kv, int num_sms, int* out);
 cudaError_t score_init_attrs();
 cudaError_t topk_init_attrs();
 cudaError_t refresh_init_attrs();
+cudaError_t fp8_init_attrs();
+cudaError_t launch_score_fp8(const lsa_dims& d, const SeqTable& tab, int max_n, int n_layers, int n_heads,
+                             int mean, const uint8_t* ckv, const uint8_t* q8, const float* q_scale,
+                             const float* head_w, float* scores, uint32_t* err, cudaStream_t stream,
+                             bool pdl);
 int refresh_max_chunks();
 cudaError_t launch_refresh(const lsa_dims& d, const SeqTable& tab, int max_n, const int32_t* new_ids,
                            int32_t* slot_ids, const void* K, const void* V, void* K_res, void* V_res,
@@ -63,7 +68,7 @@ lsa_status device_info(DeviceInfo* out) {
         di.sms = sms;
         // kernel attributes are per device: set them here, never inside a launch (graph capture)
         if (score_init_attrs() != cudaSuccess || topk_init_attrs() != cudaSuccess ||
-            refresh_init_attrs() != cudaSuccess)
+            refresh_init_attrs() != cudaSuccess || fp8_init_attrs() != cudaSuccess)
             return LSA_ERR_CUDA;
         if (attn_ctas_per_device(LSA_F32, sms, &di.attn_ctas[LSA_F32]) != cudaSuccess) return LSA_ERR_CUDA;
         if (attn_ctas_per_device(LSA_BF16, sms, &di.attn_ctas[LSA_BF16]) != cudaSuccess) return LSA_ERR_CUDA;
@@ -325,6 +330,67 @@ lsa_status lsa_decode_step_threshold(const lsa_dims* dims, const void* q_emb, co
         e = launch_attention(*dims, p.tab, di.attn_ctas[dims->kv_dtype], q, K, V, chunk_ids_out,
                              reinterpret_cast<float*>(at(ws, w.part_o)),
                              reinterpret_cast<float*>(at(ws, w.part_ml)), out, lse, err, st, true, kept_count_out);
+    return cuda_status(e);
+}
+
+namespace {
+lsa_status check_fp8_args(const lsa_dims* d, int32_t n_layers, int32_t n_heads, lsa_ensemble ens,
+                          const void* ckv, const void* q8, const float* q_scale, const float* head_w) {
+    if (d->E != LSA_INDEX_DIM) return LSA_ERR_INVALID_ARG;
+    if (n_layers < 1 || n_layers > 16) return LSA_ERR_INVALID_ARG;
+    if (n_heads < 16 || n_heads > 256 || n_heads % 16 != 0) return LSA_ERR_UNSUPPORTED;
+    if (ens != LSA_ENSEMBLE_MAX && ens != LSA_ENSEMBLE_MEAN) return LSA_ERR_INVALID_ARG;
+    if (!aligned16(ckv) || !aligned16(q8)) return LSA_ERR_INVALID_ARG;
+    if (q_scale == nullptr || head_w == nullptr || (reinterpret_cast<uintptr_t>(q_scale) & 3u) ||
+        (reinterpret_cast<uintptr_t>(head_w) & 3u))
+        return LSA_ERR_INVALID_ARG;
+    return LSA_OK;
+}
+}  // namespace
+
+lsa_status lsa_indexer_score_fp8(const lsa_dims* dims, int32_t n_layers, int32_t n_heads, lsa_ensemble ensemble,
+                                 const void* compressed_k, const void* q_fp8, const float* q_scale,
+                                 const float* head_w, float* scores, void* ws, size_t ws_bytes, void* stream) {
+    Prepared p;
+    DeviceInfo di;
+    WsLayout w;
+    lsa_status s = prepare_ws(dims, ws, ws_bytes, &p, &di, &w);
+    if (s != LSA_OK) return s;
+    s = check_fp8_args(dims, n_layers, n_heads, ensemble, compressed_k, q_fp8, q_scale, head_w);
+    if (s != LSA_OK) return s;
+    if (!aligned16(scores)) return LSA_ERR_INVALID_ARG;
+    return cuda_status(launch_score_fp8(*dims, p.tab, p.max_n, n_layers, n_heads, ensemble == LSA_ENSEMBLE_MEAN,
+                                        static_cast<const uint8_t*>(compressed_k), static_cast<const uint8_t*>(q_fp8),
+                                        q_scale, head_w, scores, reinterpret_cast<uint32_t*>(ws),
+                                        static_cast<cudaStream_t>(stream), false));
+}
+
+lsa_status lsa_decode_step_fp8(const lsa_dims* dims, int32_t n_layers, int32_t n_heads, lsa_ensemble ensemble,
+                               const void* compressed_k, const void* q_fp8, const float* q_scale,
+                               const float* head_w, const void* q, const void* K, const void* V,
+                               int32_t* chunk_ids_out, float* out, float* lse, void* ws, size_t ws_bytes,
+                               void* stream) {
+    Prepared p;
+    DeviceInfo di;
+    WsLayout w;
+    lsa_status s = prepare_ws(dims, ws, ws_bytes, &p, &di, &w);
+    if (s != LSA_OK) return s;
+    s = check_fp8_args(dims, n_layers, n_heads, ensemble, compressed_k, q_fp8, q_scale, head_w);
+    if (s != LSA_OK) return s;
+    if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(chunk_ids_out) || !aligned16(out))
+        return LSA_ERR_INVALID_ARG;
+    if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LSA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+    float* scores = reinterpret_cast<float*>(at(ws, w.scores));
+    cudaError_t e = launch_score_fp8(*dims, p.tab, p.max_n, n_layers, n_heads, ensemble == LSA_ENSEMBLE_MEAN,
+                                     static_cast<const uint8_t*>(compressed_k), static_cast<const uint8_t*>(q_fp8),
+                                     q_scale, head_w, scores, err, st, false);
+    if (e == cudaSuccess) e = launch_topk(*dims, p.tab, p.max_n, scores, chunk_ids_out, err, st, true);
+    if (e == cudaSuccess)
+        e = launch_attention(*dims, p.tab, di.attn_ctas[dims->kv_dtype], q, K, V, chunk_ids_out,
+                             reinterpret_cast<float*>(at(ws, w.part_o)),
+                             reinterpret_cast<float*>(at(ws, w.part_ml)), out, lse, err, st, true);
     return cuda_status(e);
 }
 

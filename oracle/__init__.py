@@ -18,7 +18,9 @@ dimensionstp.github.io, section 3-2 (2)-(3); arXiv abstract):
 5. footprint = k * chunk_len / L;
 6. the retrieval cycle's resident refresh (review section 3-1 "retrieval interval" and
    section 3-2 (3) step 7): the slot table after a cycle, written out as its rule;
-7. the threshold keep mask with a fallback floor (section 3-2 (3) step 5).
+7. the threshold keep mask with a fallback floor (section 3-2 (3) step 5);
+8. the indexer score on FP8 compressed-K chunks (section 3-2 (1)-(2)), decoding the
+   132-byte chunk format and float8_e4m3 from their definitions.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (hand-worked fixtures in ``tests/golden/``, closed forms, a brute-force
@@ -52,6 +54,8 @@ def _load():
         lib.lsa_oracle_attention.restype = None
         lib.lsa_oracle_footprint.argtypes = [i64, i64, i64]
         lib.lsa_oracle_footprint.restype = ctypes.c_double
+        lib.lsa_oracle_indexer_scores.argtypes = [i64, i64, i64, i64, ctypes.c_int, dp, dp, dp, dp, dp, dp]
+        lib.lsa_oracle_indexer_scores.restype = None
         _lib = lib
     return _lib
 
@@ -173,3 +177,41 @@ def threshold_select(scores, tau: float, k_min: int, k_max: int) -> np.ndarray:
     count = int(np.count_nonzero(s >= float(tau)))
     k_eff = min(max(count, min(int(k_min), int(k_max))), int(k_max))
     return topk(s, k_eff)
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """float8_e4m3 (the "fn" variant: no infinities) bit patterns -> exact float64.
+
+    1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits; exponent 0 is subnormal
+    (m/8 * 2^-6); the all-ones exponent with mantissa 7 is NaN, the other codes with
+    exponent 15 are normal numbers (up to 448)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c >> 7 == 1, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    normal = (1.0 + m / 8.0) * np.power(2.0, e - 7)
+    sub = (m / 8.0) * 2.0 ** -6
+    val = sign * np.where(e == 0, sub, normal)
+    return np.where((e == 15) & (m == 7), np.nan, val)
+
+
+def split_compressed_k(rows) -> tuple:
+    """132-byte compressed-K rows (review section 3-2 (1)): bytes 0..127 are e4m3 key values,
+    bytes 128..131 a little-endian float32 dequant scale. Returns (keys float64, scales float64)."""
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.uint8))
+    assert r.shape[-1] == 132
+    keys = e4m3_decode(r[..., :128])
+    scales = r[..., 128:132].copy().view("<f4")[..., 0].astype(np.float64)
+    return keys, scales
+
+
+def indexer_scores(k, ks, q, qs, w, mean: bool = False) -> np.ndarray:
+    """s_i = ens_l sigmoid(sum_h w_lh ReLU(ks_li qs_lh q_lh . k_li)) for one sequence.
+    k [L][n][D], ks [L][n], q [L][H][D], qs [L][H], w [L][H] (float64 values)."""
+    k, ks, q, qs, w = _f64(k), _f64(ks), _f64(q), _f64(qs), _f64(w)
+    L, n, D = k.shape
+    H = q.shape[1]
+    s = np.empty(n, dtype=np.float64)
+    _load().lsa_oracle_indexer_scores(n, L, H, D, 1 if mean else 0, _dp(k), _dp(ks), _dp(q), _dp(qs),
+                                      _dp(w), _dp(s))
+    return s

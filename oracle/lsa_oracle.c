@@ -142,3 +142,38 @@ double lsa_oracle_footprint(int64_t k, int64_t chunk_len, int64_t context_len)
 {
     return (double)(k * chunk_len) / (double)context_len;
 }
+
+/*
+ * Neural Memory Indexer score on compressed-K chunks (review section 3-2 (2): per-head
+ * queries q_h, chunk key k_i, fused head weights w_h, sigmoid of the ReLU-weighted sum;
+ * section 3-2 (2): the per-layer scores are ensembled by max or mean). Inputs are the
+ * dequantised values' factors: keys k [L][n][D] with per-chunk scales ks [L][n], queries
+ * q [L][H][D] with per-head scales qs [L][H], weights w [L][H]. For every chunk i:
+ *     v_l = sum_h w[l][h] * max(0, ks[l][i] * qs[l][h] * sum_d q[l][h][d] * k[l][i][d])
+ *     s_l = 1 / (1 + exp(-v_l))
+ *     s[i] = max_l s_l   (mean = 0)   or   (1/L) sum_l s_l   (mean = 1)
+ */
+void lsa_oracle_indexer_scores(int64_t n, int64_t L, int64_t H, int64_t D, int mean,
+                               const double *k, const double *ks, const double *q,
+                               const double *qs, const double *w, double *s)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        double comb = mean ? 0.0 : -INFINITY;
+        for (int64_t l = 0; l < L; ++l) {
+            double v = 0.0;
+            for (int64_t h = 0; h < H; ++h) {
+                double dot = 0.0;
+                for (int64_t d = 0; d < D; ++d)
+                    dot += q[(l * H + h) * D + d] * k[(l * n + i) * D + d];
+                double a = ks[l * n + i] * qs[l * H + h] * dot;
+                v += w[l * H + h] * (a > 0.0 ? a : 0.0);
+            }
+            double sl = 1.0 / (1.0 + exp(-v));
+            if (mean)
+                comb += sl;
+            else if (sl > comb)
+                comb = sl;
+        }
+        s[i] = mean ? comb / (double)L : comb;
+    }
+}

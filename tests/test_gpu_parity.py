@@ -469,3 +469,68 @@ def test_decode_step_threshold(lsa, case):
             G.check_ids(mine, ref, s, k_eff)
         ref_o, _ = G.oracle_attention(dw, b, mine)
         np.testing.assert_allclose(out[b], ref_o, rtol=0, atol=1e-4)
+
+
+# ------------------------------------------------------------------ FP8 compressed-K indexer score
+FP8_CASES = [
+    dict(B=2, N=(300, 129), L=3, Hn=128, mean=False),
+    dict(B=1, N=(64,), L=1, Hn=16, mean=True),
+    dict(B=3, N=(257, 1, 128), L=2, Hn=64, mean=False),
+    dict(B=2, N=(130, 400), L=3, Hn=256, mean=True),
+]
+
+
+@pytest.mark.parametrize("case", FP8_CASES, ids=lambda c: f"B{c['B']}-L{c['L']}-H{c['Hn']}-{'mean' if c['mean'] else 'max'}")
+def test_indexer_score_fp8_parity(lsa, case):
+    w = datagen.small_workload(B=case["B"], N=case["N"], k=[1] * case["B"], E=128, emb_dtype="bf16",
+                               kv_dtype="bf16", seed=77)
+    ix = G.IndexerInputs(w, case["L"], case["Hn"], case["mean"])
+    dims = G.dims_of(w, lsa)
+    ws = lsa.alloc_workspace(dims)
+    sc = torch.empty(w.total_chunks, dtype=torch.float32, device="cuda")
+    lsa.lsa_indexer_score_fp8(dims, case["L"], case["Hn"], int(case["mean"]), ix.ck, ix.q8, ix.qs, ix.hw, sc, ws)
+    assert lsa.lsa_get_device_status(ws) == lsa.LSA_OK
+    got = sc.cpu().numpy().astype(np.float64)
+    off = w.chunk_offsets
+    worst = 0.0
+    for b in range(w.B):
+        ref, tol = ix.oracle_scores(b), ix.tolerance(b)
+        err = np.abs(got[off[b]:off[b + 1]] - ref)
+        worst = max(worst, float((err / tol).max()))
+        assert (err <= tol).all(), f"max err {err.max()} vs tol {tol[err.argmax()]}"
+    print(f"fp8 indexer: worst error / tolerance = {worst:.3g}")
+
+
+def test_indexer_fp8_full_size_1m(lsa):
+    # the 1M-context shape: 16384 chunks, 3 layers, 128 heads
+    w = datagen.Workload("1m-idx", 1, [16384], 128, 1, [2212], 16, seed=3, plant="copy", plant_count=[164])
+    ix = G.IndexerInputs(w, 3, 128)
+    dims = G.dims_of(w, lsa)
+    ws = lsa.alloc_workspace(dims)
+    sc = torch.empty(w.total_chunks, dtype=torch.float32, device="cuda")
+    lsa.lsa_indexer_score_fp8(dims, 3, 128, lsa.LSA_ENSEMBLE_MAX, ix.ck, ix.q8, ix.qs, ix.hw, sc, ws)
+    ids = torch.empty(2212, dtype=torch.int32, device="cuda")
+    lsa.lsa_topk_select(dims, sc, ids, ws)
+    assert lsa.lsa_get_device_status(ws) == lsa.LSA_OK
+    ref, tol = ix.oracle_scores(0), ix.tolerance(0)
+    got = sc.cpu().numpy().astype(np.float64)
+    assert (np.abs(got - ref) <= tol).all()
+    G.check_ids(ids.cpu().numpy(), oracle.topk(ref, 2212), ref, 2212, band=float(tol.max()))
+    assert set(datagen.planted_positions(w, 0).tolist()) <= set(ids.cpu().numpy().tolist())
+
+
+def test_decode_step_fp8(lsa):
+    w = datagen.small_workload(B=2, N=(300, 129), k=(40, 13), E=128, H=16, emb_dtype="bf16", kv_dtype="bf16",
+                               seed=78)
+    dw = G.DeviceWorkload(w, lsa)
+    ix = G.IndexerInputs(w, 3, 128)
+    lsa.lsa_decode_step_fp8(dw.dims, 3, 128, lsa.LSA_ENSEMBLE_MAX, ix.ck, ix.q8, ix.qs, ix.hw, dw.q, dw.K, dw.V,
+                            dw.ids, dw.out, dw.lse, dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_OK
+    got, out = dw.ids.cpu().numpy(), dw.out.cpu().numpy()
+    for b in range(w.B):
+        ref, tol = ix.oracle_scores(b), ix.tolerance(b)
+        mine = got[w.k_offsets[b]:w.k_offsets[b + 1]]
+        G.check_ids(mine, oracle.topk(ref, w.k[b]), ref, w.k[b], band=float(tol.max()))
+        ref_o, _ = G.oracle_attention(dw, b, mine)
+        np.testing.assert_allclose(out[b], ref_o, rtol=0, atol=1e-4)

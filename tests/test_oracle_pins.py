@@ -315,3 +315,43 @@ def test_threshold_properties():
         else:                                    # cap: all kept chunks pass
             assert (s[ids] >= tau).all()
         np.testing.assert_array_equal(ids, oracle.topk(s, len(ids)))  # always a top-k set
+
+
+# ---------------------------------------------------------------- FP8 indexer score
+def test_indexer_golden():
+    g = load("indexer_score.txt")
+    k = g["k"].reshape(2, 2, 2)
+    q = g["q"].reshape(2, 2, 2)
+    for mean, key in ((False, "s_max"), (True, "s_mean")):
+        s = oracle.indexer_scores(k, g["ks"], q, g["qs"], g["w"], mean=mean)
+        np.testing.assert_allclose(s, g[key], rtol=0, atol=1e-15)
+
+
+def test_e4m3_decode_matches_library():
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_decode(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    np.testing.assert_array_equal(np.isnan(ours), np.isnan(ref))
+    np.testing.assert_array_equal(ours[~np.isnan(ours)], ref[~np.isnan(ref)])
+    assert oracle.e4m3_decode([0x7E])[0] == 448.0 and oracle.e4m3_decode([0x01])[0] == 2.0 ** -9
+
+
+def test_compressed_k_split():
+    row = np.zeros((1, 132), dtype=np.uint8)
+    row[0, :3] = [0x38, 0xC0, 0x01]                      # 1.0, -2.0, 2^-9
+    row[0, 128:] = np.array([0.75], dtype="<f4").view(np.uint8)
+    keys, scales = oracle.split_compressed_k(row)
+    np.testing.assert_array_equal(keys[0, :4], [1.0, -2.0, 2.0 ** -9, 0.0])
+    assert scales[0] == 0.75
+
+
+def test_indexer_reduces_to_dot_product():
+    # one layer, one head, weight 1, unit scales, a positive dot: s = sigmoid(q . k)
+    rng = np.random.default_rng(14)
+    q, k = rng.standard_normal((1, 1, 8)), rng.standard_normal((1, 5, 8))
+    k[0] *= np.sign(k[0] @ q[0, 0])[:, None]              # make every dot positive
+    s = oracle.indexer_scores(k, np.ones((1, 5)), q, np.ones((1, 1)), np.ones((1, 1)))
+    np.testing.assert_allclose(s, 1.0 / (1.0 + np.exp(-(k[0] @ q[0, 0]))), rtol=0, atol=1e-15)
+    # ReLU: a negative head contributes nothing
+    s0 = oracle.indexer_scores(-k, np.ones((1, 5)), q, np.ones((1, 1)), np.ones((1, 1)))
+    np.testing.assert_allclose(s0, 0.5, rtol=0, atol=0)
