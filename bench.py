@@ -381,6 +381,9 @@ def run_ours(args):
                "gbs_per_gpu": S.step_bytes() * K / (ms / 1e3) / 1e9, "bytes_per_step": S.step_bytes()}
         res["frac_of_measured"] = res["gbs_per_gpu"] / peak
         res["frac_of_spec_8tbs"] = res["gbs_per_gpu"] / SPEC_HBM_GBS
+        if name == "1m":
+            # the pages' own indexer score (FP8 compressed-K, 3 layers x 128 heads) feeding the same step
+            res["fp8_indexer_step"] = fp8_step_loop(S, K, W, world)
         if name == args.workload:
             head = S
             # the dominant kernel alone: split-K attention (+ its merge) over the last step's kept ids
@@ -490,6 +493,49 @@ def e2e_loop(S, K: int, W: int, world: int) -> dict:
     bo = h_out.numel() * h_out.element_size() + h_ids.numel() * h_ids.element_size()
     return {"value": K / (ms / 1e3) * world, "unit": "steps/s", "h2d_bytes_per_step": bi,
             "d2h_bytes_per_step": bo, "ms_per_step": ms / K}
+
+
+def fp8_step_loop(S, K: int, W: int, world: int, layers: int = 3, heads: int = 128) -> dict:
+    """Steps/s of lsa_decode_step_fp8: FP8 compressed-K indexer score -> top-k -> attention."""
+    import torch
+
+    import datagen
+    w, lsa = S.w, S.lsa
+    x = datagen.make_indexer_inputs(w, layers, heads)
+    ck = torch.from_numpy(x["compressed_k"]).cuda()
+    q8 = torch.from_numpy(x["q_fp8"]).cuda()
+    qs = torch.from_numpy(x["q_scale"]).cuda()
+    hw = torch.from_numpy(x["head_w"]).cuda()
+    R = len(S.q)
+    dims = lsa.Dims(w.B, 1, lsa.LSA_INDEX_DIM, w.H, w.C, N=w.N[0], k=w.k[0], emb_dtype="bf16",
+                    kv_dtype=w.kv_dtype)
+
+    def step(r):
+        lsa.lsa_decode_step_fp8(dims, layers, heads, lsa.LSA_ENSEMBLE_MAX, ck, q8, qs, hw, S.q[r], S.K, S.V,
+                                S.ids, S.out, S.lse, S.ws)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for r in range(R):
+            step(r)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graphs = []
+    for r in range(R):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(r)
+        graphs.append(g)
+    ms = time_loop(lambda i: graphs[i % R].replay(), K, W, world)
+    st = lsa.lsa_get_device_status(S.ws)
+    if st != lsa.LSA_OK:
+        raise SystemExit(f"device error in the fp8 step: {lsa.string(st)}")
+    kv = w.esize("kv_dtype")
+    step_bytes = (ck.numel() + q8.numel() + 4 * (qs.numel() + hw.numel())
+                  + w.total_kept * w.C * w.H * w.Dh * kv * 2 + w.B * w.H * w.Dh * (kv + 4) + w.total_kept * 4)
+    return {"layers": layers, "heads": heads, "steps_per_s": K / (ms / 1e3) * world, "ms_per_step": ms / K,
+            "gbs": step_bytes * K / (ms / 1e3) / 1e9 * world, "bytes_per_step": step_bytes}
 
 
 def interval_loop(S, K: int, W: int, world: int, every: int = 64) -> dict:

@@ -238,6 +238,53 @@ LSA_API lsa_status lsa_decode_step_fp8(const lsa_dims *dims, int32_t n_layers, i
                                        const void *V, int32_t *chunk_ids_out, float *out, float *lse, void *ws,
                                        size_t ws_bytes, void *stream);
 
+/* Sparse decode attention over a per-sequence device count of kept chunks: as
+ * lsa_sparse_decode_attn with chunk_ids (the capacity k_b from dims), attending over the
+ * first kept_count[b] ids only (kept_count [B] int32 device, 0 <= count <= k_b). A count of 0
+ * gives out = 0 and lse = -inf. */
+LSA_API lsa_status lsa_sparse_decode_attn_counts(const lsa_dims *dims, const void *q, const void *K,
+                                                 const void *V, const int32_t *chunk_ids,
+                                                 const int32_t *kept_count, float *out, float *lse, void *ws,
+                                                 size_t ws_bytes, void *stream);
+
+/* Chunk-sharded step across G ranks (this library's multi-GPU form of [R3-2.3 steps 4-7]:
+ * a sequence's chunks are split into contiguous runs, one per rank). Per rank:
+ *   1. lsa_score_chunks and lsa_topk_select on its own chunks with k_local = min(k, n_local);
+ *   2. lsa_shard_candidates -> (score, global id) candidates, padded to k_pad with
+ *      (-FLT_MAX, -1); the caller all-gathers them into [G][B][k_pad];
+ *   3. lsa_shard_global_select -> the global keep set (the top-k of the candidates, ties to
+ *      the lower global id) and this rank's share of it (local ids + count);
+ *   4. lsa_sparse_decode_attn_counts over its share -> (out_g, lse_g); the caller all-gathers
+ *      them into [G][B][H][Dh] and [G][B][H];
+ *   5. lsa_merge_partials -> the step's output (log-sum-exp merge).
+ * Scores must be greater than -FLT_MAX. */
+
+/* Step 2. local_dims: this rank's shard (k / k_per_seq = its local candidate counts);
+ * local_ids [sum k_local] from lsa_topk_select; global_offset host [B]: global id of the
+ * rank's first chunk per sequence; cand_scores [B][k_pad] float32 and cand_ids [B][k_pad]
+ * int32, out. */
+LSA_API lsa_status lsa_shard_candidates(const lsa_dims *local_dims, const float *scores, const int32_t *local_ids,
+                                        const int32_t *global_offset, int32_t k_pad, float *cand_scores,
+                                        int32_t *cand_ids, void *stream);
+
+/* Step 3. global_dims: B, N = G * k_pad, k / k_per_seq = the global k (no chunk_offsets);
+ * global_offset, local_n host [B]: this rank's first global chunk id and chunk count per
+ * sequence; all_scores [G][B][k_pad], all_ids [G][B][k_pad]: the gathered candidates;
+ * seq_scores, seq_ids [B][G*k_pad]: caller scratch; global_ids [sum k] out (nullable): the
+ * global keep set, ascending; local_ids [sum_b min(k_b, local_n_b)] out: this rank's kept
+ * ids (local, ascending) then -1; local_count [B] out. ws: a workspace for global_dims. */
+LSA_API lsa_status lsa_shard_global_select(const lsa_dims *global_dims, int32_t G, const int32_t *global_offset,
+                                           const int32_t *local_n, const float *all_scores, const int32_t *all_ids,
+                                           float *seq_scores, int32_t *seq_ids, int32_t *global_ids,
+                                           int32_t *local_ids, int32_t *local_count, void *ws, size_t ws_bytes,
+                                           void *stream);
+
+/* Step 5. outs [G][B][H][Dh] float32 normalised outputs, lses [G][B][H] natural-log sums
+ * (-inf for a rank that kept nothing); out [B][H][Dh], lse [B][H] (nullable):
+ *   out = sum_g e^(lse_g - M) out_g / sum_g e^(lse_g - M),  lse = M + log sum_g e^(lse_g - M). */
+LSA_API lsa_status lsa_merge_partials(int32_t G, int32_t B, int32_t H, const float *outs, const float *lses,
+                                      float *out, float *lse, void *stream);
+
 /* Synchronise `stream`, read the sticky device error word of `ws`, clear it, and
  * return LSA_OK or the first device error (NONFINITE, BAD_ID, TIMEOUT, in that order). */
 LSA_API lsa_status lsa_get_device_status(void *ws, void *stream);

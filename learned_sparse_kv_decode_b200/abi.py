@@ -69,6 +69,12 @@ def _load():
                                   ctypes.c_int),
         "lsa_decode_step_fp8": ([dp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp,
                                  vp, vp, vp, sz, vp], ctypes.c_int),
+        "lsa_sparse_decode_attn_counts": ([dp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+        "lsa_shard_candidates": ([dp, vp, vp, ctypes.POINTER(ctypes.c_int32), ctypes.c_int32, vp, vp, vp],
+                                 ctypes.c_int),
+        "lsa_shard_global_select": ([dp, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32),
+                                     vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+        "lsa_merge_partials": ([ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, vp, vp, vp, vp, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -203,6 +209,35 @@ def lsa_decode_step_threshold(dims, q_emb, chunk_emb, q, K, V, tau, k_min, chunk
     _check(lib.lsa_decode_step_threshold(dims.ptr, _p(q_emb), _p(chunk_emb), _p(q), _p(K), _p(V), float(tau),
                                          int(k_min), _p(chunk_ids_out), _p(kept_count_out), _p(out), _p(lse),
                                          _p(ws), _nbytes(ws), _stream(stream)), "lsa_decode_step_threshold")
+
+
+def _i32(values):
+    return (ctypes.c_int32 * len(values))(*map(int, values))
+
+
+def lsa_sparse_decode_attn_counts(dims, q, K, V, chunk_ids, kept_count, out, lse, ws, stream=None) -> None:
+    _check(lib.lsa_sparse_decode_attn_counts(dims.ptr, _p(q), _p(K), _p(V), _p(chunk_ids), _p(kept_count), _p(out),
+                                             _p(lse), _p(ws), _nbytes(ws), _stream(stream)),
+           "lsa_sparse_decode_attn_counts")
+
+
+def lsa_shard_candidates(local_dims, scores, local_ids, global_offset, k_pad, cand_scores, cand_ids,
+                         stream=None) -> None:
+    _check(lib.lsa_shard_candidates(local_dims.ptr, _p(scores), _p(local_ids), _i32(global_offset), int(k_pad),
+                                    _p(cand_scores), _p(cand_ids), _stream(stream)), "lsa_shard_candidates")
+
+
+def lsa_shard_global_select(global_dims, G, global_offset, local_n, all_scores, all_ids, seq_scores, seq_ids,
+                            global_ids, local_ids, local_count, ws, stream=None) -> None:
+    _check(lib.lsa_shard_global_select(global_dims.ptr, int(G), _i32(global_offset), _i32(local_n), _p(all_scores),
+                                       _p(all_ids), _p(seq_scores), _p(seq_ids), _p(global_ids), _p(local_ids),
+                                       _p(local_count), _p(ws), _nbytes(ws), _stream(stream)),
+           "lsa_shard_global_select")
+
+
+def lsa_merge_partials(G, B, H, outs, lses, out, lse, stream=None) -> None:
+    _check(lib.lsa_merge_partials(int(G), int(B), int(H), _p(outs), _p(lses), _p(out), _p(lse), _stream(stream)),
+           "lsa_merge_partials")
 
 
 def lsa_refresh_resident(dims, q_emb, chunk_emb, K, V, slot_ids, K_res, V_res, moved, ws, stream=None) -> None:

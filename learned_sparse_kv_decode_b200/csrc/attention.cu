@@ -363,6 +363,11 @@ k_attn_merge(const float* __restrict__ part_o, const float* __restrict__ part_ml
     float M = s_red[0];
 #pragma unroll
     for (int w = 1; w < kMergeThreads / 32; ++w) M = fmaxf(M, s_red[w]);
+    if (M == -INFINITY) {  // no kept token at all (a count of 0): empty output, lse = -inf
+        if (threadIdx.x < kMergeDims) out[((uint64_t)b * ap.H + h) * kDh + blockIdx.z * kMergeDims + threadIdx.x] = 0.f;
+        if (lse != nullptr && threadIdx.x == 0 && blockIdx.z == 0) lse[(uint64_t)b * ap.H + h] = -INFINITY;
+        return;
+    }
     // 2. slot weights 2^(m_s - M) and the merged denominator L
     float lloc = 0.f;
     for (int i = tid; i < ns; i += kMergeThreads) {

@@ -26,6 +26,19 @@ cudaError_t score_init_attrs();
 cudaError_t topk_init_attrs();
 cudaError_t refresh_init_attrs();
 cudaError_t fp8_init_attrs();
+struct ShardOffsets {
+    int32_t global0[kMaxB];
+};
+cudaError_t launch_shard_candidates(const SeqTable& tab, int B, const ShardOffsets& offs, int k_pad,
+                                    const float* scores, const int32_t* ids, float* cs, int32_t* ci,
+                                    cudaStream_t st);
+cudaError_t launch_shard_transpose(int G, int B, int k_pad, const float* in_s, const int32_t* in_i, float* out_s,
+                                   int32_t* out_i, cudaStream_t st);
+cudaError_t launch_shard_select(const int32_t* pos, const int32_t* cand_ids, const SeqTable& gtab,
+                                const ShardOffsets& offs, const SeqTable& ltab, int B, int G, int k_pad,
+                                int32_t* local_ids, int32_t* local_count, int32_t* global_ids, cudaStream_t st);
+cudaError_t launch_merge_partials(const float* outs, const float* lses, int G, int B, int H, float* out, float* lse,
+                                  cudaStream_t st);
 cudaError_t launch_score_fp8(const lsa_dims& d, const SeqTable& tab, int max_n, int n_layers, int n_heads,
                              int mean, const uint8_t* ckv, const uint8_t* q8, const float* q_scale,
                              const float* head_w, float* scores, uint32_t* err, cudaStream_t stream,
@@ -392,6 +405,99 @@ lsa_status lsa_decode_step_fp8(const lsa_dims* dims, int32_t n_layers, int32_t n
                              reinterpret_cast<float*>(at(ws, w.part_o)),
                              reinterpret_cast<float*>(at(ws, w.part_ml)), out, lse, err, st, true);
     return cuda_status(e);
+}
+
+lsa_status lsa_sparse_decode_attn_counts(const lsa_dims* dims, const void* q, const void* K, const void* V,
+                                         const int32_t* chunk_ids, const int32_t* kept_count, float* out,
+                                         float* lse, void* ws, size_t ws_bytes, void* stream) {
+    Prepared p;
+    DeviceInfo di;
+    WsLayout w;
+    lsa_status s = prepare_ws(dims, ws, ws_bytes, &p, &di, &w);
+    if (s != LSA_OK) return s;
+    if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(chunk_ids) || !aligned16(kept_count) ||
+        !aligned16(out))
+        return LSA_ERR_INVALID_ARG;
+    if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LSA_ERR_INVALID_ARG;
+    return cuda_status(launch_attention(*dims, p.tab, di.attn_ctas[dims->kv_dtype], q, K, V, chunk_ids,
+                                        reinterpret_cast<float*>(at(ws, w.part_o)),
+                                        reinterpret_cast<float*>(at(ws, w.part_ml)), out, lse,
+                                        reinterpret_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream), false,
+                                        kept_count));
+}
+
+lsa_status lsa_shard_candidates(const lsa_dims* local_dims, const float* scores, const int32_t* local_ids,
+                                const int32_t* global_offset, int32_t k_pad, float* cand_scores,
+                                int32_t* cand_ids, void* stream) {
+    Prepared p;
+    lsa_status s = prepare(local_dims, &p);
+    if (s != LSA_OK) return s;
+    if (global_offset == nullptr || !aligned16(scores) || !aligned16(local_ids) || !aligned16(cand_scores) ||
+        !aligned16(cand_ids))
+        return LSA_ERR_INVALID_ARG;
+    ShardOffsets offs;
+    std::memset(&offs, 0, sizeof(offs));
+    for (int b = 0; b < local_dims->B; ++b) {
+        const int kb = p.tab.kept_off[b + 1] - p.tab.kept_off[b];
+        if (global_offset[b] < 0 || kb > k_pad) return LSA_ERR_INVALID_ARG;
+        offs.global0[b] = global_offset[b];
+    }
+    if (k_pad < 1) return LSA_ERR_INVALID_ARG;
+    return cuda_status(launch_shard_candidates(p.tab, local_dims->B, offs, k_pad, scores, local_ids, cand_scores,
+                                               cand_ids, static_cast<cudaStream_t>(stream)));
+}
+
+lsa_status lsa_shard_global_select(const lsa_dims* global_dims, int32_t G, const int32_t* global_offset,
+                                   const int32_t* local_n, const float* all_scores, const int32_t* all_ids,
+                                   float* seq_scores, int32_t* seq_ids, int32_t* global_ids, int32_t* local_ids,
+                                   int32_t* local_count, void* ws, size_t ws_bytes, void* stream) {
+    Prepared gp;
+    DeviceInfo di;
+    WsLayout w;
+    lsa_status s = prepare_ws(global_dims, ws, ws_bytes, &gp, &di, &w);
+    if (s != LSA_OK) return s;
+    if (global_dims->chunk_offsets != nullptr || G < 1 || global_dims->N % G != 0) return LSA_ERR_INVALID_ARG;
+    if (global_offset == nullptr || local_n == nullptr || !aligned16(all_scores) || !aligned16(all_ids) ||
+        !aligned16(seq_scores) || !aligned16(seq_ids) || !aligned16(local_ids) || !aligned16(local_count) ||
+        (global_ids != nullptr && !aligned16(global_ids)))
+        return LSA_ERR_INVALID_ARG;
+    const int k_pad = global_dims->N / G;
+    const int B = global_dims->B;
+    // this rank's local table: its chunk counts, and one slot per globally kept chunk as capacity
+    SeqTable ltab;
+    std::memset(&ltab, 0, sizeof(ltab));
+    ltab.B = B;
+    ltab.C = global_dims->chunk_len;
+    ShardOffsets offs;
+    std::memset(&offs, 0, sizeof(offs));
+    int64_t chunks = 0, cap = 0;
+    for (int b = 0; b < B; ++b) {
+        if (local_n[b] < 1 || global_offset[b] < 0) return LSA_ERR_INVALID_ARG;
+        const int kb = gp.tab.kept_off[b + 1] - gp.tab.kept_off[b];
+        ltab.chunk_off[b] = (int32_t)chunks;
+        ltab.kept_off[b] = (int32_t)cap;
+        chunks += local_n[b];
+        cap += kb < local_n[b] ? kb : local_n[b];  // a rank keeps at most min(k, its chunks)
+        offs.global0[b] = global_offset[b];
+    }
+    ltab.chunk_off[B] = (int32_t)chunks;
+    ltab.kept_off[B] = (int32_t)cap;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t* pos = reinterpret_cast<int32_t*>(at(ws, w.ids));
+    cudaError_t e = launch_shard_transpose(G, B, k_pad, all_scores, all_ids, seq_scores, seq_ids, st);
+    if (e == cudaSuccess)
+        e = launch_topk(*global_dims, gp.tab, gp.max_n, seq_scores, pos, reinterpret_cast<uint32_t*>(ws), st, false);
+    if (e == cudaSuccess)
+        e = launch_shard_select(pos, seq_ids, gp.tab, offs, ltab, B, G, k_pad, local_ids, local_count, global_ids, st);
+    return cuda_status(e);
+}
+
+lsa_status lsa_merge_partials(int32_t G, int32_t B, int32_t H, const float* outs, const float* lses, float* out,
+                              float* lse, void* stream) {
+    if (G < 1 || B < 1 || H < 1 || H > 65535 || B > 65535) return LSA_ERR_INVALID_ARG;
+    if (!aligned16(outs) || !aligned16(lses) || !aligned16(out)) return LSA_ERR_INVALID_ARG;
+    if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LSA_ERR_INVALID_ARG;
+    return cuda_status(launch_merge_partials(outs, lses, G, B, H, out, lse, static_cast<cudaStream_t>(stream)));
 }
 
 lsa_status lsa_refresh_resident(const lsa_dims* dims, const void* q_emb, const void* chunk_emb,

@@ -14,6 +14,7 @@ import datagen
 import oracle
 from datagen import device as dgdev
 from tests import _gpu as G
+from tests import _gpu as GPU  # the same module, for tests where G is a rank count
 
 pytestmark = pytest.mark.gpu
 
@@ -534,3 +535,48 @@ def test_decode_step_fp8(lsa):
         G.check_ids(mine, oracle.topk(ref, w.k[b]), ref, w.k[b], band=float(tol.max()))
         ref_o, _ = G.oracle_attention(dw, b, mine)
         np.testing.assert_allclose(out[b], ref_o, rtol=0, atol=1e-4)
+
+
+# ------------------------------------------------------------------ chunk-sharded step (emulated ranks)
+SHARD_CASES = [
+    dict(B=2, N=(300, 129), k=(40, 13), E=128, H=16, emb_dtype="bf16", kv_dtype="bf16", G=2),
+    dict(B=2, N=(300, 129), k=(40, 13), E=128, H=16, emb_dtype="bf16", kv_dtype="bf16", G=4),
+    dict(B=1, N=(600,), k=(81,), E=256, Q=64, H=16, emb_dtype="bf16", kv_dtype="bf16", plant="copy_query", G=3),
+    dict(B=2, N=(64, 90), k=(1, 1), E=64, H=8, emb_dtype="f32", kv_dtype="f32", G=4),  # most ranks keep nothing
+]
+
+
+@pytest.mark.parametrize("case", SHARD_CASES, ids=lambda c: f"G{c['G']}-B{c['B']}-Q{c.get('Q', 1)}-k{c['k'][0]}")
+def test_sharded_step_emulated(lsa, case):
+    from learned_sparse_kv_decode_b200 import sharded
+    case = dict(case)
+    G = case.pop("G")
+    w = datagen.small_workload(seed=88, **case)
+    dw = GPU.DeviceWorkload(w, lsa)
+    off = w.chunk_offsets
+    backends, embs, Ks, Vs = [], [], [], []
+    for g, (ln, go) in enumerate(sharded.split_chunks(w.N, G)):
+        plan = sharded.ShardPlan(w.B, w.Q, w.E, w.H, w.C, G, g, w.k, ln, go, w.emb_dtype, w.kv_dtype)
+        backends.append(sharded.CudaShardBackend(plan))
+        embs.append(torch.cat([dw.chunk_emb[off[b] + go[b]:off[b] + go[b] + ln[b]] for b in range(w.B)]).contiguous())
+        Ks.append(torch.cat([dw.K[(off[b] + go[b]) * w.C:(off[b] + go[b] + ln[b]) * w.C] for b in range(w.B)]).contiguous())
+        Vs.append(torch.cat([dw.V[(off[b] + go[b]) * w.C:(off[b] + go[b] + ln[b]) * w.C] for b in range(w.B)]).contiguous())
+    results, gids = sharded.run_emulated(backends, dw.q_emb, embs, dw.q, Ks, Vs)
+    # the unsharded fused step on the same inputs
+    lsa.lsa_decode_step(dw.dims, dw.q_emb, dw.chunk_emb, dw.q, dw.K, dw.V, dw.ids, dw.out, dw.lse, dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_OK
+    for bk in backends:
+        assert lsa.lsa_get_device_status(bk.ws_local) == lsa.LSA_OK
+        assert lsa.lsa_get_device_status(bk.ws_global) == lsa.LSA_OK
+    np.testing.assert_array_equal(gids.cpu().numpy(), dw.ids.cpu().numpy())  # identical fp32 scores
+    ref_out = dw.out.cpu().numpy()
+    for out, lse in results:
+        np.testing.assert_allclose(out.cpu().numpy(), ref_out, rtol=0, atol=1e-4)
+        np.testing.assert_allclose(lse.cpu().numpy(), dw.lse.cpu().numpy(), rtol=0, atol=1e-4)
+    got = gids.cpu().numpy()
+    for b in range(w.B):
+        ref_s = oracle.chunk_scores(dw.q_emb_f(b), dw.emb_f(b))
+        mine = got[w.k_offsets[b]:w.k_offsets[b + 1]]
+        GPU.check_ids(mine, oracle.topk(ref_s, w.k[b]), ref_s, w.k[b])
+        ref_o, _ = GPU.oracle_attention(dw, b, mine)
+        np.testing.assert_allclose(results[0][0][b].cpu().numpy(), ref_o, rtol=0, atol=1e-4)
