@@ -381,7 +381,7 @@ def run_ours(args):
                "gbs_per_gpu": S.step_bytes() * K / (ms / 1e3) / 1e9, "bytes_per_step": S.step_bytes()}
         res["frac_of_measured"] = res["gbs_per_gpu"] / peak
         res["frac_of_spec_8tbs"] = res["gbs_per_gpu"] / SPEC_HBM_GBS
-        if name == "1m":
+        if name in ("1m", "1m-h2"):
             # the pages' own indexer score (FP8 compressed-K, 3 layers x 128 heads) feeding the same step
             res["fp8_indexer_step"] = fp8_step_loop(S, K, W, world)
         if name == args.workload:

@@ -13,10 +13,12 @@
 //     v_il = sum_h w_lh * ReLU(ks_li * qs_blh * (q8_blh . k8_li)),  s_il = 1 / (1 + e^-v_il)
 // and s_i = max_l s_il (or the mean).
 //
-// Per CTA: 128 chunks of one sequence. For each layer, the 128 x 132-byte rows are read
-// with coalesced 4-byte loads and split into the fp8 keys (written straight into the
+// Per CTA: 128 chunks of one sequence. For each layer, the 128 x 132-byte rows arrive by one
+// 1-D bulk copy (16-byte aligned window, a tail of < 16 bytes by plain loads) into a
+// double-buffered raw tile and are re-laid out in shared memory into the fp8 keys (the
 // no-swizzle K-major core-matrix layout) and the scales; the queries of all heads arrive by
-// 2-D TMA tile loads into the same layout. One tcgen05 MMA chain of kind::f8f6f4
+// 2-D TMA tile loads into the same layout. The next layer loads while this one computes.
+// One tcgen05 MMA chain of kind::f8f6f4
 // (M = 128 chunks, N = heads, K = 128 in 4 steps of 32) accumulates q8 . k8 in TMEM
 // (fp32); the epilogue reads a row per thread (tcgen05.ld) and applies scales, ReLU,
 // head weights and the sigmoid.
@@ -58,17 +60,22 @@ __device__ __forceinline__ void idx_tma_2d(uint32_t dst, const CUtensorMap* map,
         : "memory");
 }
 
+// Bytes of one raw tile buffer: up to 128 rows of 132 bytes plus 12 bytes of alignment slack.
+constexpr int kIdxRawBytes = (kIdxM * kIdxRowBytes + 16 + 15) / 16 * 16;
+
 // grid (ceil(maxN/128), B), 128 threads.
-// dynamic smem: A keys [8 K-chunks][128 rows][16 B] | B queries [8][Hn][16 B] | key scales [128]
-//               | query scales [Hn] | head weights [Hn]
-// ckv: compressed keys [L][sum N][132]; tmQ: e4m3 queries [B*L*Hn rows][128], box 16 x Hn.
+// dynamic smem: A keys [8 K-chunks][128 rows][16 B] | B queries [2][8][Hn][16 B] (double buffer)
+//               | raw rows [2][kIdxRawBytes] (double buffer) | key scales [128] | query scales [Hn]
+//               | head weights [Hn]
+// ckv: compressed keys [L][sum N][132] (ckv_bytes long); tmQ: e4m3 queries [B*L*Hn rows][128],
+// box 16 x Hn. Layer l+1's rows and queries load (1-D bulk copy + 2-D TMA) while layer l runs.
 __global__ void __launch_bounds__(128)
-k_score_fp8(const uint8_t* __restrict__ ckv, const __grid_constant__ CUtensorMap tmQ,
+k_score_fp8(const uint8_t* __restrict__ ckv, uint64_t ckv_bytes, const __grid_constant__ CUtensorMap tmQ,
             const float* __restrict__ q_scale, const float* __restrict__ head_w,
             float* __restrict__ scores, const SeqTable tab, int n_layers, int Hn, int mean,
             int64_t total_chunks, uint32_t tmem_cols, uint32_t* err) {
     extern __shared__ __align__(1024) uint8_t smem[];
-    __shared__ __align__(8) uint64_t load_bar;
+    __shared__ __align__(8) uint64_t load_bar[2];
     __shared__ __align__(8) uint64_t mma_bar;
     __shared__ uint32_t tmem_slot;
 
@@ -80,18 +87,51 @@ k_score_fp8(const uint8_t* __restrict__ ckv, const __grid_constant__ CUtensorMap
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int rows = min(kIdxM, n_b - r0);
 
+    const uint32_t qbytes = (uint32_t)Hn * kIdxDim;
     const uint32_t sA = smem_u32(smem);
-    const uint32_t sB = sA + kIdxM * kIdxDim;
-    float* ks = reinterpret_cast<float*>(smem + kIdxM * kIdxDim + Hn * kIdxDim);
+    const uint32_t sB0 = sA + kIdxM * kIdxDim;
+    uint8_t* raw0 = smem + kIdxM * kIdxDim + 2 * qbytes;
+    float* ks = reinterpret_cast<float*>(raw0 + 2 * kIdxRawBytes);
     float* qs = ks + kIdxM;
     float* hw = qs + Hn;
-    uint32_t* a_words = reinterpret_cast<uint32_t*>(smem);
+
+    // byte window of layer l's rows: a 16-byte aligned bulk part plus a tail of < 16 bytes
+    auto window = [&](int l, uint64_t& start_al, uint32_t& delta, uint32_t& bulk, uint32_t& tail) {
+        const uint64_t off = ((uint64_t)l * total_chunks + (uint64_t)tab.chunk_off[b] + r0) * kIdxRowBytes;
+        const uint64_t end = off + (uint64_t)rows * kIdxRowBytes;
+        start_al = off & ~15ull;
+        delta = (uint32_t)(off - start_al);
+        uint64_t bulk_end = (end + 15) & ~15ull;
+        const uint64_t cap = ckv_bytes & ~15ull;
+        if (bulk_end > cap) bulk_end = cap;
+        bulk = (uint32_t)(bulk_end - start_al);
+        tail = (uint32_t)(end > bulk_end ? end - bulk_end : 0);
+    };
+    auto issue = [&](int l) {  // one thread: rows and queries of layer l into buffer l & 1
+        const int buf = l & 1;
+        uint64_t start_al;
+        uint32_t delta, bulk, tail;
+        window(l, start_al, delta, bulk, tail);
+        const uint32_t bar = smem_u32(&load_bar[buf]);
+        mbar_arrive_expect_tx(bar, bulk + qbytes);
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                smem_u32(raw0 + buf * kIdxRawBytes)),
+            "l"(ckv + start_al), "r"(bulk), "r"(bar)
+            : "memory");
+        const int row = (b * n_layers + l) * Hn;
+        const uint32_t sB = sB0 + buf * qbytes;
+        for (int c = 0; c < kIdxKChunks; ++c) idx_tma_2d(sB + (uint32_t)c * Hn * 16, &tmQ, c * 16, row, bar);
+    };
 
     if (tid == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQ)) : "memory");
-        mbar_init(smem_u32(&load_bar), 1);
+        mbar_init(smem_u32(&load_bar[0]), 1);
+        mbar_init(smem_u32(&load_bar[1]), 1);
         mbar_init(smem_u32(&mma_bar), 1);
         fence_mbar_init();
+        issue(0);
+        if (n_layers > 1) issue(1);
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -108,72 +148,61 @@ k_score_fp8(const uint8_t* __restrict__ ckv, const __grid_constant__ CUtensorMap
 
     float combined = mean ? 0.f : -INFINITY;
     bool ok = true;
-    for (int l = 0; l < n_layers && ok; ++l) {
-        // ---- queries of all heads of (b, l): TMA into the core-matrix layout
-        if (tid == 0) {
-            const uint32_t lb = smem_u32(&load_bar);
-            mbar_arrive_expect_tx(lb, (uint32_t)Hn * kIdxDim);
-            const int row = (b * n_layers + l) * Hn;
-            for (int c = 0; c < kIdxKChunks; ++c) idx_tma_2d(sB + (uint32_t)c * Hn * 16, &tmQ, c * 16, row, lb);
-        }
+    for (int l = 0; l < n_layers; ++l) {
+        const int buf = l & 1;
+        uint8_t* raw = raw0 + buf * kIdxRawBytes;
+        uint64_t start_al;
+        uint32_t delta, bulk, tail;
+        window(l, start_al, delta, bulk, tail);
         for (int h = tid; h < Hn; h += 128) {
             qs[h] = q_scale[((size_t)b * n_layers + l) * Hn + h];
             hw[h] = head_w[(size_t)l * Hn + h];
         }
-        // ---- keys: coalesced 4-byte loads of the 132-byte rows, split into keys and scales
-        const uint32_t* src = reinterpret_cast<const uint32_t*>(
-            ckv + ((size_t)l * total_chunks + (size_t)tab.chunk_off[b] + r0) * kIdxRowBytes);
-        const int words = rows * (kIdxRowBytes / 4);
-        for (int w0 = 0; w0 < kIdxM * (kIdxRowBytes / 4); w0 += 128 * 4) {
-            uint32_t v[4];
+        const bool landed = mbar_wait(smem_u32(&load_bar[buf]), (uint32_t)((l >> 1) & 1), err);
+        if (tid < (int)(tail / 4))  // the last < 16 bytes of the tensor, past the aligned bulk part
+            reinterpret_cast<uint32_t*>(raw + bulk)[tid] = __ldg(reinterpret_cast<const uint32_t*>(ckv + start_al + bulk) + tid);
+        ok = __syncthreads_and(landed) != 0;
+        if (!ok) break;
+        // re-layout: row r's 128 key bytes -> 8 core-matrix rows of 16 bytes; its scale -> ks[r]
+        {
+            const int r = tid;
+            const uint32_t* src = reinterpret_cast<const uint32_t*>(raw + delta) + r * (kIdxRowBytes / 4);
+            uint32_t w[kIdxRowBytes / 4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int wi = w0 + u * 128 + tid;
-                v[u] = wi < words ? __ldg(src + wi) : 0u;
-            }
+            for (int i = 0; i < kIdxRowBytes / 4; ++i) w[i] = r < rows ? src[i] : 0u;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int wi = w0 + u * 128 + tid;
-                if (wi >= kIdxM * (kIdxRowBytes / 4)) continue;
-                const int r = wi / (kIdxRowBytes / 4), x = wi % (kIdxRowBytes / 4);
-                if (x < kIdxDim / 4) {
-                    // byte 4x of the row: K-chunk x / 4, word x % 4 of that chunk's 16 bytes
-                    a_words[((x >> 2) * kIdxM + r) * 4 + (x & 3)] = v[u];
-                } else {
-                    ks[r] = __uint_as_float(v[u]);
-                }
-            }
+            for (int c = 0; c < kIdxKChunks; ++c)
+                *reinterpret_cast<uint4*>(smem + (c * kIdxM + r) * 16) =
+                    make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+            ks[r] = __uint_as_float(w[kIdxDim / 4]);
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // keys -> tensor core
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         __syncthreads();
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         if (tid == 0) {
-            bool loaded = mbar_wait(smem_u32(&load_bar), (uint32_t)(l & 1), err);
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            if (loaded) {
-                for (int ksx = 0; ksx < kIdxDim / 32; ++ksx) {
-                    // K-step ksx covers K-chunks 2ksx and 2ksx+1 (32 e4m3 values)
-                    const uint64_t ad = idx_desc(sA + (uint32_t)ksx * 2 * kIdxM * 16, kIdxM * 16, 128);
-                    const uint64_t bd = idx_desc(sB + (uint32_t)ksx * 2 * Hn * 16, (uint32_t)Hn * 16, 128);
-                    const uint32_t accum = ksx > 0 ? 1u : 0u;
-                    asm volatile(
-                        "{\n\t.reg .pred p;\n\t"
-                        "setp.ne.b32 p, %4, 0;\n\t"
-                        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-                        "l"(ad), "l"(bd), "r"(idesc), "r"(accum)
-                        : "memory");
-                }
+            const uint32_t sB = sB0 + buf * qbytes;
+            for (int ksx = 0; ksx < kIdxDim / 32; ++ksx) {
+                // K-step ksx covers K-chunks 2ksx and 2ksx+1 (32 e4m3 values)
+                const uint64_t ad = idx_desc(sA + (uint32_t)ksx * 2 * kIdxM * 16, kIdxM * 16, 128);
+                const uint64_t bd = idx_desc(sB + (uint32_t)ksx * 2 * Hn * 16, (uint32_t)Hn * 16, 128);
+                const uint32_t accum = ksx > 0 ? 1u : 0u;
                 asm volatile(
-                    "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                        smem_u32(&mma_bar))
+                    "{\n\t.reg .pred p;\n\t"
+                    "setp.ne.b32 p, %4, 0;\n\t"
+                    "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+                    "l"(ad), "l"(bd), "r"(idesc), "r"(accum)
                     : "memory");
-            } else {
-                mbar_arrive(smem_u32(&mma_bar));
             }
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                             smem_u32(&mma_bar))
+                         : "memory");
         }
         const bool done = mbar_wait(smem_u32(&mma_bar), (uint32_t)(l & 1), err);
         ok = __syncthreads_and(done) != 0;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         if (!ok) break;
+        if (tid == 0 && l + 2 < n_layers) issue(l + 2);  // this buffer is free: prefetch two layers ahead
 
         // ---- epilogue: row 32*warp + lane; v = sum_h w_h ReLU(ks qs_h D[row][h]); sigmoid
         const float kscale = ks[warp * 32 + lane];
@@ -198,7 +227,7 @@ k_score_fp8(const uint8_t* __restrict__ ckv, const __grid_constant__ CUtensorMap
         const float s_l = 1.f / (1.f + expf(-v));
         combined = mean ? combined + s_l : fmaxf(combined, s_l);
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        __syncthreads();  // TMEM, keys and query smem are reused by the next layer
+        __syncthreads();  // TMEM, keys and scales are reused by the next layer
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     }
     if (ok) {
@@ -213,7 +242,9 @@ k_score_fp8(const uint8_t* __restrict__ ckv, const __grid_constant__ CUtensorMap
     }
 }
 
-size_t fp8_score_smem(int Hn) { return (size_t)kIdxM * kIdxDim + (size_t)Hn * kIdxDim + (kIdxM + 2 * Hn) * 4; }
+size_t fp8_score_smem(int Hn) {
+    return (size_t)kIdxM * kIdxDim + 2 * (size_t)Hn * kIdxDim + 2 * (size_t)kIdxRawBytes + (kIdxM + 2 * Hn) * 4;
+}
 
 cudaError_t fp8_init_attrs() { return set_smem_attrs(k_score_fp8, (int)fp8_score_smem(256)); }
 
@@ -256,8 +287,9 @@ cudaError_t launch_score_fp8(const lsa_dims& d, const SeqTable& tab, int max_n, 
     cfg.gridDim = dim3((max_n + kIdxM - 1) / kIdxM, d.B, 1);
     cfg.blockDim = dim3(128, 1, 1);
     cfg.dynamicSmemBytes = fp8_score_smem(n_heads);
-    return cudaLaunchKernelEx(&cfg, k_score_fp8, ckv, tmQ, q_scale, head_w, scores, tab, n_layers, n_heads, mean,
-                              (int64_t)tab.chunk_off[d.B], cols, err);
+    const uint64_t ckv_bytes = (uint64_t)n_layers * (uint64_t)tab.chunk_off[d.B] * kIdxRowBytes;
+    return cudaLaunchKernelEx(&cfg, k_score_fp8, ckv, ckv_bytes, tmQ, q_scale, head_w, scores, tab, n_layers, n_heads,
+                              mean, (int64_t)tab.chunk_off[d.B], cols, err);
 }
 
 }  // namespace lsa
