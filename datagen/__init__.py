@@ -43,7 +43,7 @@ import numpy as np
 __all__ = [
     "GAMMA", "mix64", "stream_key", "normal_f32", "uniform_f64", "bf16_bits",
     "bf16_to_f32", "Workload", "workload", "WORKLOADS", "make_inputs",
-    "kv_rows", "TENSOR_IDS",
+    "kv_rows", "TENSOR_IDS", "make_lookahead_queries",
 ]
 
 _M64 = np.uint64(0xFFFFFFFFFFFFFFFF)
@@ -336,6 +336,17 @@ def make_query_variant(w: Workload, r: int) -> dict:
     q_emb = normal_f32(seed, TENSOR_IDS["q_emb"], np.arange(w.B * w.Q * w.E)).reshape(w.B, w.Q, w.E)
     q = normal_f32(seed, TENSOR_IDS["q"], np.arange(w.B * w.H * w.Dh)).reshape(w.B, w.H, w.Dh)
     return {"q_emb": _store(q_emb, w.emb_dtype), "q": _store(q, w.kv_dtype)}
+
+
+TENSOR_IDS["q_la"] = 17  # attention queries of the lookahead window [B, Q, H, Dh]
+
+
+def make_lookahead_queries(w: Workload, seed: int | None = None) -> np.ndarray:
+    """Attention queries of the Q-token lookahead window, [B, Q, H, Dh], in the K/V storage
+    type: element (b, j, h, d) is element ((b*Q + j)*H + h)*Dh + d of stream 'q_la'."""
+    s = w.seed if seed is None else seed
+    q = normal_f32(s, TENSOR_IDS["q_la"], np.arange(w.B * w.Q * w.H * w.Dh)).reshape(w.B, w.Q, w.H, w.Dh)
+    return _store(q, w.kv_dtype)
 
 
 TENSOR_IDS.update({"idx_q": 11, "idx_k": 12, "idx_qs": 13, "idx_ks": 14, "idx_w": 15, "idx_plant": 16})

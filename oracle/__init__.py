@@ -20,7 +20,9 @@ dimensionstp.github.io, section 3-2 (2)-(3); arXiv abstract):
    section 3-2 (3) step 7): the slot table after a cycle, written out as its rule;
 7. the threshold keep mask with a fallback floor (section 3-2 (3) step 5);
 8. the indexer score on FP8 compressed-K chunks (section 3-2 (1)-(2)), decoding the
-   132-byte chunk format and float8_e4m3 from their definitions.
+   132-byte chunk format and float8_e4m3 from their definitions;
+9. the lookahead window's attention: every one of the window's queries attends over the
+   same kept tokens (section 3-2 (3)), one ordinary decode attention per query.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (hand-worked fixtures in ``tests/golden/``, closed forms, a brute-force
@@ -109,6 +111,25 @@ def attention(q, K, V, scale: float | None = None):
     return out, lse
 
 
+def lookahead_attention(q, K, V, scale: float | None = None):
+    """Attention of every query of the lookahead window over the same kept tokens.
+
+    The indexer keeps the chunks that the next ~64 tokens will attend to, and until the next
+    retrieval cycle each of those tokens attends over the kept chunks (review on
+    dimensionstp.github.io, section 3-2 (3), lookahead window and steps 6-7). Read plainly:
+    query j of the window is an ordinary decode query over the kept set, with no mask
+    between the window's queries. q [Q, H, Dh]; K, V [T, H, Dh].
+    Returns (out [Q, H, Dh], lse [Q, H]); row j is ``attention(q[j], K, V, scale)``."""
+    q = _f64(q)
+    assert q.ndim == 3
+    outs, lses = [], []
+    for j in range(q.shape[0]):
+        o, l = attention(q[j], K, V, scale)
+        outs.append(o)
+        lses.append(l)
+    return np.stack(outs), np.stack(lses)
+
+
 def kept_tokens(ids, chunk_len: int) -> np.ndarray:
     """Token positions (within the sequence) covered by the kept chunks, in kept order."""
     ids = np.asarray(ids, dtype=np.int64)
@@ -136,6 +157,19 @@ def decode_step(q_emb, chunk_emb, q, K, V, k: int, chunk_len: int, scale: float 
     Kk = K(tok) if callable(K) else np.asarray(K)[tok]
     Vk = V(tok) if callable(V) else np.asarray(V)[tok]
     out, lse = attention(q, Kk, Vk, scale)
+    return ids, out, lse, s
+
+
+def decode_step_lookahead(q_emb, chunk_emb, q, K, V, k: int, chunk_len: int, scale: float | None = None):
+    """One sequence's step for the whole lookahead window: scores (max over the Q query
+    embeddings) -> top-k -> gather -> every window query's attention over the kept tokens.
+    q is [Q, H, Dh]. Returns (ids, out [Q, H, Dh], lse [Q, H], scores)."""
+    s = chunk_scores(q_emb, chunk_emb)
+    ids = topk(s, k)
+    tok = kept_tokens(ids, chunk_len)
+    Kk = K(tok) if callable(K) else np.asarray(K)[tok]
+    Vk = V(tok) if callable(V) else np.asarray(V)[tok]
+    out, lse = lookahead_attention(q, Kk, Vk, scale)
     return ids, out, lse, s
 
 

@@ -67,3 +67,14 @@ def test_make_inputs_tiny_planting():
     pos = datagen.planted_positions(w, 0)
     d = x["chunk_emb"][pos] - x["q_emb"][0, 0][None, :]
     assert float(np.abs(d).max()) < 0.1 * 6.0 + 1e-6
+
+
+def test_lookahead_queries_layout_and_storage():
+    w = datagen.small_workload(Q=5, H=3, kv_dtype="bf16")
+    x = datagen.make_lookahead_queries(w)
+    assert x.shape == (w.B, 5, 3, w.Dh) and x.dtype == np.uint16
+    b, j, h, d = 1, 4, 2, 77
+    idx = ((b * w.Q + j) * w.H + h) * w.Dh + d
+    v = datagen.normal_f32(w.seed, datagen.TENSOR_IDS["q_la"], np.array([idx]))[0]
+    assert x[b, j, h, d] == datagen.bf16_bits(np.array([v], np.float32))[0]
+    assert datagen.TENSOR_IDS["q_la"] not in [t for k, t in datagen.TENSOR_IDS.items() if k != "q_la"]

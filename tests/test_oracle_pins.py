@@ -151,6 +151,57 @@ def test_sparse_attention_equals_masked_dense():
     np.testing.assert_allclose(out, _sdpa(q, K, V, mask), rtol=0, atol=1e-13)
 
 
+# ---------------------------------------------------------------- lookahead window attention
+def test_lookahead_golden_two_queries():
+    g = load("lookahead_two_queries.txt")
+    q = g["q"].reshape(2, 2, 4)
+    K, V = g["K"].reshape(2, 2, 4), g["V"].reshape(2, 2, 4)
+    out, lse = oracle.lookahead_attention(q, K, V)
+    np.testing.assert_allclose(out.reshape(4, 4), g["out"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse.reshape(4), g["lse"], rtol=0, atol=1e-15)
+
+
+def test_lookahead_matches_library_multi_query_sdpa():
+    # every window query over every kept token, no mask between the queries: one library
+    # call with a query length of Q
+    rng = np.random.default_rng(9)
+    Qw, T, H, Dh = 64, 200, 3, 128
+    q = rng.standard_normal((Qw, H, Dh))
+    K, V = rng.standard_normal((T, H, Dh)), rng.standard_normal((T, H, Dh))
+    out, lse = oracle.lookahead_attention(q, K, V)
+    qt = torch.from_numpy(q).permute(1, 0, 2)                       # [H, Q, Dh]
+    Kt, Vt = torch.from_numpy(K).permute(1, 0, 2), torch.from_numpy(V).permute(1, 0, 2)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt).permute(1, 0, 2).numpy()
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-13)
+    z = torch.einsum("hqd,htd->hqt", qt, Kt) / math.sqrt(Dh)
+    np.testing.assert_allclose(lse, torch.logsumexp(z, dim=-1).permute(1, 0).numpy(), rtol=0, atol=1e-12)
+
+
+def test_lookahead_equivariance():
+    rng = np.random.default_rng(10)
+    Qw, T, H, Dh = 7, 50, 2, 16
+    q = rng.standard_normal((Qw, H, Dh))
+    K, V = rng.standard_normal((T, H, Dh)), rng.standard_normal((T, H, Dh))
+    out, lse = oracle.lookahead_attention(q, K, V)
+    pq, pt = rng.permutation(Qw), rng.permutation(T)
+    out2, lse2 = oracle.lookahead_attention(q[pq], K[pt], V[pt])
+    np.testing.assert_allclose(out2, out[pq], rtol=0, atol=1e-13)   # queries permute the rows
+    np.testing.assert_allclose(lse2, lse[pq], rtol=0, atol=1e-13)   # tokens do not matter in order
+
+
+def test_lookahead_step_with_one_query_is_the_decode_step():
+    rng = np.random.default_rng(11)
+    n, E, H, Dh, C, k = 30, 16, 2, 8, 4, 6
+    q_emb, emb = rng.standard_normal((1, E)), rng.standard_normal((n, E))
+    q = rng.standard_normal((H, Dh))
+    K, V = rng.standard_normal((n * C, H, Dh)), rng.standard_normal((n * C, H, Dh))
+    ids, out, lse, s = oracle.decode_step(q_emb, emb, q, K, V, k, C)
+    ids2, out2, lse2, s2 = oracle.decode_step_lookahead(q_emb, emb, q[None], K, V, k, C)
+    np.testing.assert_array_equal(ids, ids2)
+    np.testing.assert_array_equal(out, out2[0])
+    np.testing.assert_array_equal(lse, lse2[0])
+
+
 def test_attention_single_token_returns_v():
     rng = np.random.default_rng(6)
     q, K, V = rng.standard_normal((3, 128)), rng.standard_normal((1, 3, 128)), rng.standard_normal((1, 3, 128))
