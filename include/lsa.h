@@ -178,6 +178,32 @@ LSA_API lsa_status lsa_decode_step(const lsa_dims *dims, const void *q_emb, cons
                            int32_t *chunk_ids_out, float *out, float *lse,
                            void *ws, size_t ws_bytes, void *stream);
 
+/* Attention of every query of the lookahead window over the kept tokens [R3-2.3: the indexer
+ * keeps the chunks that the next ~64 tokens will attend to; steps 6-7]. Each of the
+ * dims->Q window queries is an independent decode query over the same kept set, with no
+ * mask between the window's queries:
+ *   q         [B][Q][H][Dh] bf16, the window's attention queries (Q = dims->Q, 1..64)
+ *   K, V      bf16; chunk_ids != NULL: the full caches [sum L_b][H][Dh] read through the ids;
+ *             chunk_ids == NULL: resident buffers [sum k_b*C][H][Dh]
+ *   out       [B][Q][H][Dh] float32: softmax(q_j . K^T / sqrt(Dh)) V over the kept tokens
+ *   lse       [B][Q][H] float32 natural-log sums, or NULL
+ * kv_dtype must be LSA_BF16 and Q <= 64 (else LSA_ERR_UNSUPPORTED); the token rows of K/V
+ * must number below 2^31. A tcgen05 flash-attention kernel: S = Q.K^T and O += P.V on the
+ * tensor cores (bf16 operands, fp32 accumulation, P rounded to bf16), online softmax in fp32,
+ * split-K over one SM-balanced tile list with a log-sum-exp merge. */
+LSA_API lsa_status lsa_sparse_decode_attn_lookahead(const lsa_dims *dims, const void *q, const void *K,
+                                                    const void *V, const int32_t *chunk_ids, float *out,
+                                                    float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/* The fused lookahead step: score with the window's Q query embeddings (max over them) ->
+ * top-k -> every window query's attention over the kept chunks [R3-2.3 steps 4-7].
+ * q_emb [B][Q][E]; q [B][Q][H][Dh] bf16; other arguments as lsa_decode_step and
+ * lsa_sparse_decode_attn_lookahead. Four kernels chained with programmatic dependent launch. */
+LSA_API lsa_status lsa_decode_step_lookahead(const lsa_dims *dims, const void *q_emb, const void *chunk_emb,
+                                             const void *q, const void *K, const void *V,
+                                             int32_t *chunk_ids_out, float *out, float *lse, void *ws,
+                                             size_t ws_bytes, void *stream);
+
 /* Retrieval cycle of the lookahead loop [R3-2.3 steps 4-7; review section 3-1: the
  * indexer re-scores about every 64 decode steps and attention runs over the kept
  * chunks until the next cycle]. Scores every chunk, keeps the top-k, and refreshes a

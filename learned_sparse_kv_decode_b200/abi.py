@@ -59,6 +59,8 @@ def _load():
         "lsa_gather_kv": ([dp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "lsa_sparse_decode_attn": ([dp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "lsa_decode_step": ([dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+        "lsa_sparse_decode_attn_lookahead": ([dp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+        "lsa_decode_step_lookahead": ([dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "lsa_get_device_status": ([vp, vp], ctypes.c_int),
         "lsa_sparse_decode_attn_noalloc": ([dp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsa_refresh_resident": ([dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
@@ -183,6 +185,18 @@ def lsa_sparse_decode_attn(dims, q, K, V, chunk_ids, out, lse, ws, stream=None) 
 def lsa_decode_step(dims, q_emb, chunk_emb, q, K, V, chunk_ids_out, out, lse, ws, stream=None) -> None:
     _check(lib.lsa_decode_step(dims.ptr, _p(q_emb), _p(chunk_emb), _p(q), _p(K), _p(V), _p(chunk_ids_out),
                                _p(out), _p(lse), _p(ws), _nbytes(ws), _stream(stream)), "lsa_decode_step")
+
+
+def lsa_sparse_decode_attn_lookahead(dims, q, K, V, chunk_ids, out, lse, ws, stream=None) -> None:
+    _check(lib.lsa_sparse_decode_attn_lookahead(dims.ptr, _p(q), _p(K), _p(V), _p(chunk_ids), _p(out), _p(lse),
+                                                _p(ws), _nbytes(ws), _stream(stream)),
+           "lsa_sparse_decode_attn_lookahead")
+
+
+def lsa_decode_step_lookahead(dims, q_emb, chunk_emb, q, K, V, chunk_ids_out, out, lse, ws, stream=None) -> None:
+    _check(lib.lsa_decode_step_lookahead(dims.ptr, _p(q_emb), _p(chunk_emb), _p(q), _p(K), _p(V),
+                                         _p(chunk_ids_out), _p(out), _p(lse), _p(ws), _nbytes(ws),
+                                         _stream(stream)), "lsa_decode_step_lookahead")
 
 
 def lsa_indexer_score_fp8(dims, n_layers, n_heads, ensemble, compressed_k, q_fp8, q_scale, head_w, scores, ws,

@@ -48,6 +48,12 @@ cudaError_t launch_refresh(const lsa_dims& d, const SeqTable& tab, int max_n, co
                            int32_t* slot_ids, const void* K, const void* V, void* K_res, void* V_res,
                            int32_t* copy_src, int32_t* copy_dst, int32_t* copy_count, int32_t* moved,
                            cudaStream_t stream);
+cudaError_t la_init_attrs(int* ctas_per_sm);
+int la_max_queries();
+int64_t la_tiles(const lsa_dims& d, const SeqTable& tab);
+cudaError_t launch_attention_la(const lsa_dims& d, const SeqTable& tab, int max_ctas, const void* q, const void* K,
+                                const void* V, int64_t kv_rows, const int32_t* ids, float* part_o, float* part_ml,
+                                float* out, float* lse, uint32_t* err, cudaStream_t stream, bool pdl);
 cudaError_t launch_attention(const lsa_dims& d, const SeqTable& tab, int ctas_per_device,
                              const void* q, const void* K, const void* V, const int32_t* ids,
                              float* part_o, float* part_ml, float* out, float* lse, uint32_t* err,
@@ -64,6 +70,7 @@ struct DeviceInfo {
     bool ready;
     int sms;
     int attn_ctas[2];  // per kv dtype (LSA_F32, LSA_BF16)
+    int la_ctas;       // CTAs of the lookahead-window attention
 };
 
 std::mutex g_dev_mu;
@@ -85,6 +92,9 @@ lsa_status device_info(DeviceInfo* out) {
             return LSA_ERR_CUDA;
         if (attn_ctas_per_device(LSA_F32, sms, &di.attn_ctas[LSA_F32]) != cudaSuccess) return LSA_ERR_CUDA;
         if (attn_ctas_per_device(LSA_BF16, sms, &di.attn_ctas[LSA_BF16]) != cudaSuccess) return LSA_ERR_CUDA;
+        int la_occ = 0;
+        if (la_init_attrs(&la_occ) != cudaSuccess || la_occ < 1) return LSA_ERR_CUDA;
+        di.la_ctas = la_occ * sms;
         di.ready = true;
     }
     *out = di;
@@ -151,10 +161,14 @@ lsa_status prepare(const lsa_dims* d, Prepared* p) {
 }
 
 struct WsLayout {
-    size_t scores, part_o, part_ml, ids, copy_src, copy_dst, copy_count, total;
+    size_t scores, part_o, part_ml, ids, copy_src, copy_dst, copy_count, la_o, la_ml, total;
 };
 
-// Workspace: header (sticky error word) | scores | split partials | refresh buffers.
+// The lookahead-window attention runs for bf16 K/V and windows of up to 64 queries.
+bool la_shape(const lsa_dims* d) { return d->kv_dtype == LSA_BF16 && d->Q <= la_max_queries(); }
+
+// Workspace: header (sticky error word) | scores | split partials | refresh buffers |
+// lookahead partials.
 WsLayout ws_layout(const lsa_dims* d, const Prepared& p, const DeviceInfo& di) {
     WsLayout w;
     const int slots = di.attn_ctas[d->kv_dtype] + d->B;
@@ -165,7 +179,11 @@ WsLayout ws_layout(const lsa_dims* d, const Prepared& p, const DeviceInfo& di) {
     w.copy_src = align256(w.ids + (size_t)p.total_kept * 4);
     w.copy_dst = align256(w.copy_src + (size_t)p.total_kept * 4);
     w.copy_count = align256(w.copy_dst + (size_t)p.total_kept * 4);
-    w.total = align256(w.copy_count + (size_t)d->B * 4);
+    // lookahead partials: two slots per CTA (its first and last (sequence, head) run)
+    const size_t la_slots = la_shape(d) ? (size_t)2 * di.la_ctas : 0;
+    w.la_o = align256(w.copy_count + (size_t)d->B * 4);
+    w.la_ml = align256(w.la_o + la_slots * d->Q * LSA_HEAD_DIM * 4);
+    w.total = align256(w.la_ml + la_slots * d->Q * 2 * 4);
     return w;
 }
 
@@ -301,6 +319,73 @@ lsa_status lsa_decode_step(const lsa_dims* dims, const void* q_emb, const void* 
     e = launch_attention(*dims, p.tab, di.attn_ctas[dims->kv_dtype], q, K, V, chunk_ids_out,
                          reinterpret_cast<float*>(at(ws, w.part_o)),
                          reinterpret_cast<float*>(at(ws, w.part_ml)), out, lse, err, st, true);
+    return cuda_status(e);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Shape checks of the lookahead-window attention; rows of the K/V tensors it reads.
+lsa_status la_check(const lsa_dims* d, const Prepared& p, bool indexed, int64_t* kv_rows) {
+    if (d->kv_dtype != LSA_BF16) return LSA_ERR_UNSUPPORTED;
+    if (d->Q > la_max_queries()) return LSA_ERR_UNSUPPORTED;
+    const int64_t rows = (indexed ? p.total_chunks : p.total_kept) * (int64_t)d->chunk_len;
+    if (rows >= (1ll << 31) || la_tiles(*d, p.tab) >= (1ll << 31)) return LSA_ERR_UNSUPPORTED;
+    *kv_rows = rows;
+    return LSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lsa_status lsa_sparse_decode_attn_lookahead(const lsa_dims* dims, const void* q, const void* K, const void* V,
+                                            const int32_t* chunk_ids, float* out, float* lse, void* ws,
+                                            size_t ws_bytes, void* stream) {
+    Prepared p;
+    DeviceInfo di;
+    WsLayout w;
+    lsa_status s = prepare_ws(dims, ws, ws_bytes, &p, &di, &w);
+    if (s != LSA_OK) return s;
+    int64_t kv_rows = 0;
+    s = la_check(dims, p, chunk_ids != nullptr, &kv_rows);
+    if (s != LSA_OK) return s;
+    if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return LSA_ERR_INVALID_ARG;
+    if (chunk_ids != nullptr && !aligned16(chunk_ids)) return LSA_ERR_INVALID_ARG;
+    if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LSA_ERR_INVALID_ARG;
+    return cuda_status(launch_attention_la(*dims, p.tab, di.la_ctas, q, K, V, kv_rows, chunk_ids,
+                                           reinterpret_cast<float*>(at(ws, w.la_o)),
+                                           reinterpret_cast<float*>(at(ws, w.la_ml)), out, lse,
+                                           reinterpret_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream),
+                                           false));
+}
+
+lsa_status lsa_decode_step_lookahead(const lsa_dims* dims, const void* q_emb, const void* chunk_emb, const void* q,
+                                     const void* K, const void* V, int32_t* chunk_ids_out, float* out, float* lse,
+                                     void* ws, size_t ws_bytes, void* stream) {
+    Prepared p;
+    DeviceInfo di;
+    WsLayout w;
+    lsa_status s = prepare_ws(dims, ws, ws_bytes, &p, &di, &w);
+    if (s != LSA_OK) return s;
+    int64_t kv_rows = 0;
+    s = la_check(dims, p, true, &kv_rows);
+    if (s != LSA_OK) return s;
+    if (!aligned16(q_emb) || !aligned16(chunk_emb) || !aligned16(q) || !aligned16(K) || !aligned16(V) ||
+        !aligned16(chunk_ids_out) || !aligned16(out))
+        return LSA_ERR_INVALID_ARG;
+    if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LSA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+    float* scores = reinterpret_cast<float*>(at(ws, w.scores));
+    cudaError_t e = launch_score(*dims, p.tab, p.max_n, q_emb, chunk_emb, scores, err, di.sms, st, false);
+    if (e != cudaSuccess) return LSA_ERR_CUDA;
+    e = launch_topk(*dims, p.tab, p.max_n, scores, chunk_ids_out, err, st, true);
+    if (e != cudaSuccess) return LSA_ERR_CUDA;
+    e = launch_attention_la(*dims, p.tab, di.la_ctas, q, K, V, kv_rows, chunk_ids_out,
+                            reinterpret_cast<float*>(at(ws, w.la_o)), reinterpret_cast<float*>(at(ws, w.la_ml)),
+                            out, lse, err, st, true);
     return cuda_status(e);
 }
 

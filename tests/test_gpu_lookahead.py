@@ -1,0 +1,214 @@
+"""GPU parity of the lookahead-window attention (every window query over the kept tokens) and
+of the fused lookahead step, against the float64 oracle on the same seeded inputs.
+
+Tolerance (bf16 K/V, 2e-2 absolute on the output, as for the single-query path): the kernel
+rounds each softmax weight p to bf16 (relative error <= 2^-9) and normalises by the sum of the
+rounded weights, so the output is a convex combination whose weights are off by at most
+2 * 2^-9 relative. That bounds the error by 2^-8 * max|V| (~0.018 for these N(0,1) caches), and
+the lse by log(1 + 2^-9) < 2e-3 (4e-3 is checked to leave room for the fp32 score rounding)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import datagen
+import oracle
+from tests import _gpu as G
+
+pytestmark = pytest.mark.gpu
+
+OUT_ATOL = 2e-2
+LSE_ATOL = 4e-3
+
+
+@pytest.fixture(scope="module")
+def lsa():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import learned_sparse_kv_decode_b200 as m
+    return m
+
+
+def _free():
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+class Window:
+    """A workload on the device plus its window queries [B, Q, H, Dh] and output buffers."""
+
+    def __init__(self, w, lsa):
+        self.dw = G.DeviceWorkload(w, lsa)
+        self.q_host = datagen.make_lookahead_queries(w)
+        self.q = G.to_device(self.q_host, w.kv_dtype)
+        self.out = torch.full((w.B, w.Q, w.H, w.Dh), float("nan"), dtype=torch.float32, device="cuda")
+        self.lse = torch.full((w.B, w.Q, w.H), float("nan"), dtype=torch.float32, device="cuda")
+
+    def random_ids(self, seed):
+        rng = np.random.default_rng(seed)
+        w = self.dw.w
+        return [np.sort(rng.choice(w.N[b], size=w.k[b], replace=False)).astype(np.int32) for b in range(w.B)]
+
+    def oracle(self, b, ids, heads=None, queries=None):
+        w = self.dw.w
+        heads = np.arange(w.H) if heads is None else np.asarray(heads)
+        queries = np.arange(w.Q) if queries is None else np.asarray(queries)
+        tok = oracle.kept_tokens(ids, w.C)
+        K = self.dw.kv_f("K", b, tok, heads)
+        V = self.dw.kv_f("V", b, tok, heads)
+        q = datagen.as_f32(self.q_host[b], w.kv_dtype)[queries][:, heads]
+        return oracle.lookahead_attention(q, K, V, 1.0 / math.sqrt(w.Dh))
+
+
+def _compare(win, b, ids, heads=None, queries=None):
+    ref_o, ref_l = win.oracle(b, ids, heads, queries)
+    w = win.dw.w
+    heads = np.arange(w.H) if heads is None else np.asarray(heads)
+    queries = np.arange(w.Q) if queries is None else np.asarray(queries)
+    got_o = win.out[b].cpu().numpy()[queries][:, heads]
+    got_l = win.lse[b].cpu().numpy()[queries][:, heads]
+    assert np.isfinite(got_o).all() and np.isfinite(got_l).all()
+    np.testing.assert_allclose(got_o, ref_o, rtol=0, atol=OUT_ATOL)
+    np.testing.assert_allclose(got_l, ref_l, rtol=0, atol=LSE_ATOL)
+    return float(np.abs(got_o - ref_o).max())
+
+
+ATTN_CASES = [
+    dict(B=2, N=(40, 72), k=(5, 9), C=64, Q=64, H=4),       # runs of 5 and 9 tiles
+    dict(B=2, N=(40, 72), k=(5, 9), C=16, Q=64, H=4),       # 4 chunks a tile; ragged last tiles
+    dict(B=2, N=(30, 50), k=(7, 3), C=32, Q=64, H=2),
+    dict(B=2, N=(12, 20), k=(3, 5), C=128, Q=64, H=2),      # 2 tiles a chunk
+    dict(B=2, N=(64, 40), k=(11, 1), C=8, Q=64, H=2),       # 8 chunks a tile; a 1-chunk sequence
+    dict(B=2, N=(40, 72), k=(5, 9), C=64, Q=13, H=4),       # a partial window
+    dict(B=1, N=(40,), k=(6,), C=64, Q=1, H=8),             # a single query
+    dict(B=1, N=(2048,), k=(1024,), C=64, Q=64, H=1),       # one run split across every CTA
+    dict(B=8, N=(256,) * 8, k=(20,) * 8, C=64, Q=64, H=16),  # 128 runs: most wholly inside a CTA
+    dict(B=3, N=(300, 7, 129), k=(77, 7, 1), C=32, Q=64, H=8),
+]
+
+
+@pytest.mark.parametrize("case", ATTN_CASES,
+                         ids=lambda c: f"B{c['B']}-C{c['C']}-Q{c['Q']}-H{c['H']}-k{c['k'][0]}")
+def test_lookahead_attention_parity(lsa, case):
+    case = dict(case)
+    w = datagen.small_workload(E=64, kv_dtype="bf16", emb_dtype="bf16", seed=61, **case)
+    win = Window(w, lsa)
+    ids = win.random_ids(7)
+    ids_d = torch.from_numpy(np.concatenate(ids)).cuda()
+    lsa.lsa_sparse_decode_attn_lookahead(win.dw.dims, win.q, win.dw.K, win.dw.V, ids_d, win.out, win.lse,
+                                         win.dw.ws)
+    assert lsa.lsa_get_device_status(win.dw.ws) == lsa.LSA_OK
+    # every sequence; all heads and queries, or a sample where the oracle would be slow
+    big = w.Q * w.H * max(w.k) * w.C > 4_000_000
+    for b in range(w.B):
+        heads = sorted({0, w.H - 1}) if big else None
+        queries = sorted({0, w.Q // 2, w.Q - 1}) if big else None
+        _compare(win, b, ids[b], heads, queries)
+    del win
+    _free()
+
+
+def test_lookahead_resident_equals_indexed(lsa):
+    # the same tiles in the same order: the resident form gives bit-identical results
+    w = datagen.small_workload(B=2, N=(40, 72), k=(5, 9), C=16, E=64, Q=64, H=4, kv_dtype="bf16",
+                               emb_dtype="bf16", seed=62)
+    win = Window(w, lsa)
+    ids = torch.from_numpy(np.concatenate(win.random_ids(3))).cuda()
+    lsa.lsa_sparse_decode_attn_lookahead(win.dw.dims, win.q, win.dw.K, win.dw.V, ids, win.out, win.lse, win.dw.ws)
+    a_o, a_l = win.out.clone(), win.lse.clone()
+    rows = int(sum(w.k)) * w.C
+    K_res = torch.empty((rows, w.H, w.Dh), dtype=torch.bfloat16, device="cuda")
+    V_res = torch.empty_like(K_res)
+    lsa.lsa_gather_kv(win.dw.dims, win.dw.K, win.dw.V, ids, K_res, V_res, win.dw.ws)
+    win.out.fill_(float("nan"))
+    lsa.lsa_sparse_decode_attn_lookahead(win.dw.dims, win.q, K_res, V_res, None, win.out, win.lse, win.dw.ws)
+    assert lsa.lsa_get_device_status(win.dw.ws) == lsa.LSA_OK
+    assert torch.equal(a_o, win.out) and torch.equal(a_l, win.lse)
+
+
+def test_lookahead_one_query_matches_single_query_path(lsa):
+    # Q = 1: the window attention is the ordinary decode attention (fp32 path) up to the
+    # bf16 rounding of the softmax weights
+    w = datagen.small_workload(B=2, N=(40, 72), k=(5, 9), C=64, E=64, Q=1, H=8, kv_dtype="bf16",
+                               emb_dtype="bf16", seed=63)
+    win = Window(w, lsa)
+    ids = torch.from_numpy(np.concatenate(win.random_ids(5))).cuda()
+    lsa.lsa_sparse_decode_attn_lookahead(win.dw.dims, win.q, win.dw.K, win.dw.V, ids, win.out, win.lse, win.dw.ws)
+    q1 = win.q[:, 0].contiguous()
+    out1 = torch.empty((w.B, w.H, w.Dh), dtype=torch.float32, device="cuda")
+    lse1 = torch.empty((w.B, w.H), dtype=torch.float32, device="cuda")
+    lsa.lsa_sparse_decode_attn(win.dw.dims, q1, win.dw.K, win.dw.V, ids, out1, lse1, win.dw.ws)
+    assert lsa.lsa_get_device_status(win.dw.ws) == lsa.LSA_OK
+    torch.testing.assert_close(win.out[:, 0], out1, rtol=0, atol=OUT_ATOL)
+    torch.testing.assert_close(win.lse[:, 0], lse1, rtol=0, atol=LSE_ATOL)
+
+
+def test_lookahead_deterministic(lsa):
+    w = datagen.small_workload(B=1, N=(2048,), k=(300,), C=64, E=64, Q=64, H=2, kv_dtype="bf16",
+                               emb_dtype="bf16", seed=64)
+    win = Window(w, lsa)
+    ids = torch.from_numpy(np.concatenate(win.random_ids(9))).cuda()
+    lsa.lsa_sparse_decode_attn_lookahead(win.dw.dims, win.q, win.dw.K, win.dw.V, ids, win.out, win.lse, win.dw.ws)
+    a = (win.out.clone(), win.lse.clone())
+    for _ in range(3):
+        lsa.lsa_sparse_decode_attn_lookahead(win.dw.dims, win.q, win.dw.K, win.dw.V, ids, win.out, win.lse,
+                                             win.dw.ws)
+        assert torch.equal(a[0], win.out) and torch.equal(a[1], win.lse)
+
+
+STEP_CASES = [
+    dict(B=1, N=(600,), k=(81,), E=256, Q=64, H=16, plant="copy_query"),
+    dict(B=2, N=(130, 257), k=(18, 35), E=128, Q=64, H=4, plant="copy_query"),
+    dict(B=3, N=(40, 72, 5), k=(5, 9, 5), E=64, Q=24, H=4),
+]
+
+
+@pytest.mark.parametrize("case", STEP_CASES, ids=lambda c: f"B{c['B']}-E{c['E']}-Q{c['Q']}-H{c['H']}")
+def test_decode_step_lookahead(lsa, case):
+    w = datagen.small_workload(emb_dtype="bf16", kv_dtype="bf16", seed=65, **dict(case))
+    win = Window(w, lsa)
+    dw = win.dw
+    lsa.lsa_decode_step_lookahead(dw.dims, dw.q_emb, dw.chunk_emb, win.q, dw.K, dw.V, dw.ids, win.out, win.lse,
+                                  dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_OK
+    got = dw.ids.cpu().numpy()
+    for b in range(w.B):
+        ref_s = oracle.chunk_scores(dw.q_emb_f(b), dw.emb_f(b))
+        gids = got[w.k_offsets[b]:w.k_offsets[b + 1]]
+        G.check_ids(gids, oracle.topk(ref_s, w.k[b]), ref_s, w.k[b])
+        _compare(win, b, gids)
+
+
+def test_decode_step_lookahead_full_size_1m(lsa):
+    # the 1M lookahead workload in the launch configuration the benchmark times: all kept ids,
+    # sampled (head, query) outputs
+    w = datagen.workload("1m")
+    win = Window(w, lsa)
+    dw = win.dw
+    lsa.lsa_decode_step_lookahead(dw.dims, dw.q_emb, dw.chunk_emb, win.q, dw.K, dw.V, dw.ids, win.out, win.lse,
+                                  dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_OK
+    ref_s = oracle.chunk_scores(dw.q_emb_f(0), dw.emb_f(0))
+    gids = dw.ids.cpu().numpy()
+    G.check_ids(gids, oracle.topk(ref_s, w.k[0]), ref_s, w.k[0])
+    assert set(datagen.planted_positions(w, 0).tolist()) <= set(gids.tolist())
+    _compare(win, 0, gids, heads=[3, 12], queries=[0, 21, 63])
+    del win, dw
+    _free()
+
+
+def test_lookahead_argument_errors(lsa):
+    w = datagen.small_workload(B=1, N=(40,), k=(5,), C=64, E=64, Q=64, H=4, kv_dtype="f32", emb_dtype="bf16")
+    dw = G.DeviceWorkload(w, lsa)
+    q = torch.zeros((1, 64, 4, 128), dtype=torch.float32, device="cuda")
+    out = torch.empty((1, 64, 4, 128), dtype=torch.float32, device="cuda")
+    with pytest.raises(lsa.LsaError) as e:
+        lsa.lsa_sparse_decode_attn_lookahead(dw.dims, q, dw.K, dw.V, dw.ids, out, None, dw.ws)
+    assert e.value.status == lsa.LSA_ERR_UNSUPPORTED  # fp32 K/V: the tensor-core path is bf16
+    w2 = datagen.small_workload(B=1, N=(40,), k=(5,), C=64, E=64, Q=65, H=4, kv_dtype="bf16", emb_dtype="bf16")
+    dw2 = G.DeviceWorkload(w2, lsa)
+    q2 = torch.zeros((1, 65, 4, 128), dtype=torch.bfloat16, device="cuda")
+    out2 = torch.empty((1, 65, 4, 128), dtype=torch.float32, device="cuda")
+    with pytest.raises(lsa.LsaError) as e:
+        lsa.lsa_sparse_decode_attn_lookahead(dw2.dims, q2, dw2.K, dw2.V, dw2.ids, out2, None, dw2.ws)
+    assert e.value.status == lsa.LSA_ERR_UNSUPPORTED  # more than 64 window queries
