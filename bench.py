@@ -384,6 +384,8 @@ def run_ours(args):
         if name in ("1m", "1m-h2"):
             # the pages' own indexer score (FP8 compressed-K, 3 layers x 128 heads) feeding the same step
             res["fp8_indexer_step"] = fp8_step_loop(S, K, W, world)
+            # every query of the 64-token window attends over the kept chunks (tensor cores)
+            res["lookahead"] = lookahead_loop(S, K, W, world, peak)
         if name == args.workload:
             head = S
             # the dominant kernel alone: split-K attention (+ its merge) over the last step's kept ids
@@ -493,6 +495,59 @@ def e2e_loop(S, K: int, W: int, world: int) -> dict:
     bo = h_out.numel() * h_out.element_size() + h_ids.numel() * h_ids.element_size()
     return {"value": K / (ms / 1e3) * world, "unit": "steps/s", "h2d_bytes_per_step": bi,
             "d2h_bytes_per_step": bo, "ms_per_step": ms / K}
+
+
+def lookahead_loop(S, K: int, W: int, world: int, peak_gbs: float) -> dict:
+    """The lookahead window's attention: lsa_decode_step_lookahead (score with the Q window
+    embeddings -> top-k -> every window query over the kept chunks) as graphs over the query
+    rotations, then lsa_sparse_decode_attn_lookahead alone (its own HBM roofline)."""
+    import numpy as np
+    import torch
+
+    import datagen
+    w, lsa = S.w, S.lsa
+    R = len(S.q)
+    qla = []
+    for r in range(R):
+        a = datagen.make_lookahead_queries(w, seed=w.seed + 1000 * r)
+        qla.append(torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda())
+    out = torch.empty((w.B, w.Q, w.H, w.Dh), dtype=torch.float32, device="cuda")
+    lse = torch.empty((w.B, w.Q, w.H), dtype=torch.float32, device="cuda")
+
+    def step(r):
+        lsa.lsa_decode_step_lookahead(S.dims, S.q_emb[r], S.chunk_emb, qla[r], S.K, S.V, S.ids, out, lse, S.ws)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for r in range(R):
+            step(r)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graphs = []
+    for r in range(R):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(r)
+        graphs.append(g)
+    ms = time_loop(lambda i: graphs[i % R].replay(), K, W, world)
+    r_last = (K - 1) % R
+    ams = time_loop(lambda i: lsa.lsa_sparse_decode_attn_lookahead(S.dims, qla[r_last], S.K, S.V, S.ids, out, lse,
+                                                                   S.ws), K, W, world)
+    st = lsa.lsa_get_device_status(S.ws)
+    if st != lsa.LSA_OK:
+        raise SystemExit(f"device error in the lookahead step: {lsa.string(st)}")
+    kv = w.esize("kv_dtype")
+    tokens = w.total_kept * w.C
+    attn_bytes = (tokens * w.H * w.Dh * kv * 2 + w.B * w.Q * w.H * w.Dh * (kv + 4) + w.B * w.Q * w.H * 4
+                  + w.total_kept * 4)
+    step_bytes = attn_bytes + w.total_chunks * w.E * w.esize("emb_dtype") + w.B * w.Q * w.E * w.esize("emb_dtype")
+    flops = 4.0 * w.Q * tokens * w.H * w.Dh  # S = Q.K^T and O = P.V, useful flops
+    a_s = ams / K / 1e3
+    return {"queries": w.Q, "steps_per_s": K / (ms / 1e3) * world, "ms_per_step": ms / K,
+            "gbs": step_bytes * K / (ms / 1e3) / 1e9 * world, "bytes_per_step": step_bytes,
+            "attn_ms": ams / K, "attn_gbs": attn_bytes / a_s / 1e9, "attn_frac_of_measured": attn_bytes / a_s / 1e9 / peak_gbs,
+            "attn_bytes": attn_bytes, "attn_useful_tflops": flops / a_s / 1e12}
 
 
 def fp8_step_loop(S, K: int, W: int, world: int, layers: int = 3, heads: int = 128) -> dict:

@@ -15,26 +15,33 @@
 // One CTA per SM, persistent over a balanced run of tiles:
 //  * A tile is 64 consecutive kept tokens of one (sequence, head). The tiles of all (b, h)
 //    form one global list; CTA c takes tiles [c*S/G, (c+1)*S/G) (split-K over the list).
-//  * Warp 4 (producer) streams each tile's K and V rows from the full cache, through the
+//  * Warp 8 (producer) streams each tile's K and V rows from the full cache, through the
 //    kept chunk ids (or from a compact resident buffer), with 3-D TMA tile loads into a
 //    5-deep ring in the 128-byte-swizzled layout the MMAs read. No multicast; L2 evict-first.
-//  * Warp 5 (one thread) issues the MMAs:
-//      S  = Qd . K^T   M = 128, N = 64,  K = 128  bf16 -> fp32 TMEM, double-buffered
-//      O += P . V      M = 128, N = 128, K = 64   P from shared memory, V MN-major
+//  * Warp 9 (one thread) issues the MMAs as their inputs arrive (polling, never blocking on
+//    one barrier while another product is ready):
+//      S  = Qd . K^T   M = 128, N = 64,  K = 128  bf16 -> fp32 TMEM, 4 buffers
+//      O += P . V      M = 128, N = 128, K = 64   P read from TMEM, V an MN-major smem operand
 //    Qd holds the window's queries twice (rows 0-63 and 64-127). Rows 0-63 use the scores
 //    of the tile's tokens 0-31 and rows 64-127 those of tokens 32-63 (their P is zero over
-//    the other half). So each of the 128 softmax threads owns one (query, half-tile) row,
-//    and all four TMEM lane quarters do work. The MMAs do twice the useful flops; at 128
-//    flop per K/V byte that still sits well under the tensor-pipe roofline.
-//  * Warps 0-3 (softmax) handle one row per thread. Each thread reads its 32 scores
-//    (tcgen05.ld) and keeps a running max m and sum l in the log2 domain. It writes its bf16
-//    P row to shared memory; l sums the rounded P actually used. It rescales its O row in
-//    TMEM only when m grows by more than 8 (2^8); a stale max is exact after the final
-//    division by l.
-//  * At the end of a (b, h) run the two half-rows of each query merge in the CTA
-//    (log-sum-exp). A run wholly inside the CTA writes out/lse directly. A run split across
-//    CTAs writes a partial (O, m, l) to slot 2c (the CTA's first run) or 2c + 1 (its last
-//    run); k_attn_la_merge combines them.
+//    the other half). So each softmax thread owns one (query, half-tile) row, and all four
+//    TMEM lane quarters do work. The MMAs do twice the useful flops; at 128 flop per K/V
+//    byte that still sits well under the tensor-pipe roofline.
+//  * Warps 0-3 and 4-7 are two softmax groups that take alternate tiles. Each group has
+//    its own running max m and sum l per row (log2 domain) and its own O accumulator in
+//    TMEM, so two tiles' softmax overlap. A thread reads its 32 scores (tcgen05.ld) and
+//    writes its bf16 P row over the first 32 columns of the same S buffer (tcgen05.st); l
+//    sums the fp32 weights. It rescales its O row only when m grows by more than 8 (2^8);
+//    a stale max is exact after the final division by l.
+//  * Per S buffer, three mbarriers order the hand-offs: S landed, P written, and the O
+//    product that read P completed (the buffer is free for S four tiles later). Each
+//    completes one phase every four tiles, so no waiter can fall or run two phases out
+//    of step (a parity wait would then pass early).
+//  * At the end of a (b, h) run, group 0 merges its own and group 1's O rows straight from
+//    TMEM (same lanes), then the two half-rows of each query (log-sum-exp). A run wholly
+//    inside the CTA writes out/lse directly. A run split across CTAs writes a partial
+//    (O, m, l) to slot 2c (the CTA's first run) or 2c + 1 (its last run), and
+//    k_attn_la_merge combines them.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -56,14 +63,19 @@ constexpr uint32_t kOperand = 2 * kHalf;  // a K or V tile (16 KiB)
 constexpr uint32_t kStage = 2 * kOperand; // K + V (32 KiB)
 constexpr uint32_t kQHalf = kRows * 128;  // a 64-dim half of Qd (16 KiB)
 constexpr uint32_t kQBytes = 2 * kQHalf;  // Qd (32 KiB)
-constexpr uint32_t kPBytes = kRows * 128; // a P tile: 128 rows x 64 tokens bf16 (16 KiB)
-constexpr uint32_t kSmem = kQBytes + 2 * kPBytes + kStages * kStage + 1024;  // + alignment slack
-constexpr int kThreads = 192;             // warps 0-3 softmax, 4 producer, 5 MMA
-constexpr uint32_t kTmemCols = 256;       // S: 2 x 64 columns, then O: 128 columns
-constexpr uint32_t kTmemO = 128;          // first O column
+constexpr uint32_t kScratch = kQmax * 128 * 4;  // run-end merge: 64 rows x 128 fp32 (32 KiB)
+constexpr uint32_t kSmem = kQBytes + kScratch + kStages * kStage + 1024;  // + alignment slack
+constexpr int kThreads = 320;             // warps 0-7 softmax (two groups of 4), 8 producer, 9 MMA
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kSBufs = 4;                 // S buffers in TMEM
+constexpr uint32_t kTmemCols = 512;       // S: 4 x 64 columns, then O of group 0 and of group 1
+constexpr uint32_t kTmemO = kSBufs * kTile;  // first O column (group 0; group 1 follows)
 constexpr float kRescale = 8.0f;          // lazy-rescale threshold (log2 units)
 constexpr float kLn2 = 0.69314718055994531f;
-static_assert(kQBytes % 1024 == 0 && kPBytes % 1024 == 0 && kStage % 1024 == 0, "1 KiB swizzle atoms");
+static_assert(kQBytes % 1024 == 0 && kScratch % 1024 == 0 && kStage % 1024 == 0, "1 KiB swizzle atoms");
+static_assert(kTmemO + 2 * 128 == kTmemCols, "TMEM: S buffers then two O accumulators");
+
 }  // namespace la
 
 struct LaParams {
@@ -158,6 +170,16 @@ __device__ __forceinline__ void la_mma(uint32_t d, uint64_t a, uint64_t b, uint3
         : "memory");
 }
 
+// D (TMEM) += A (TMEM, K-major: row = lane, two bf16 per 32-bit column) . B (shared memory).
+__device__ __forceinline__ void la_mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
 __device__ __forceinline__ void la_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
@@ -181,6 +203,24 @@ __device__ __forceinline__ void la_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
           "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void la_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void la_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
 }
 
 __device__ __forceinline__ void la_st32(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -228,7 +268,21 @@ __device__ __forceinline__ float la_ex2(float x) {
     return y;
 }
 
-__device__ __forceinline__ void la_softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Non-blocking probe of an mbarrier phase (mbarrier.try_wait may suspend the thread for a while,
+// which would stall an issuer that polls several barriers).
+__device__ __forceinline__ bool la_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ void la_softmax_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // Bounded wait by a whole warp; the result is warp-uniform. Once a wait gives up (or another
 // role gave up), the CTA's roles skip their remaining waits and work but keep their barriers.
@@ -253,12 +307,14 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           const LaParams lp, uint32_t* err) {
     using namespace la;
     extern __shared__ uint8_t la_raw[];
-    __shared__ __align__(8) uint64_t bar_kf[kStages], bar_vf[kStages], bar_ke[kStages];
-    __shared__ __align__(8) uint64_t bar_sf[2], bar_pf[2], bar_od[2];
+    __shared__ __align__(8) uint64_t bar_kvf[kStages], bar_ke[kStages];  // ring stage full / empty
+    // per S buffer b: sf = S landed, pf = P written, sx = the O product reading that P has completed
+    __shared__ __align__(8) uint64_t bar_sf[kSBufs], bar_pf[kSBufs], bar_sx[kSBufs];
     __shared__ __align__(8) uint64_t bar_qf, bar_qe, bar_end;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
-    __shared__ float2 s_ml[kQmax];
+    __shared__ float2 s_ml1[kRows];  // group 1's (m, l) per row, at a run end
+    __shared__ float2 s_mlh[kQmax];  // merged (m, l) of rows 64..127, at a run end
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x;
@@ -266,21 +322,20 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const int64_t n = s1 - s0;
     const uint32_t raw = smem_u32(la_raw);
     const uint32_t sQ = (raw + 1023u) & ~1023u;
-    const uint32_t sP = sQ + kQBytes, sKV = sP + 2 * kPBytes;
-    const uint32_t kf0 = smem_u32(bar_kf), vf0 = smem_u32(bar_vf), ke0 = smem_u32(bar_ke);
-    const uint32_t sf0 = smem_u32(bar_sf), pf0 = smem_u32(bar_pf), od0 = smem_u32(bar_od);
+    const uint32_t sX = sQ + kQBytes, sKV = sX + kScratch;
+    const uint32_t kf0 = smem_u32(bar_kvf), ke0 = smem_u32(bar_ke);
+    const uint32_t sf0 = smem_u32(bar_sf), pf0 = smem_u32(bar_pf), sx0 = smem_u32(bar_sx);
     const uint32_t qf = smem_u32(&bar_qf), qe = smem_u32(&bar_qe), endb = smem_u32(&bar_end);
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(kf0 + 8 * i, 1);
-            mbar_init(vf0 + 8 * i, 1);
             mbar_init(ke0 + 8 * i, 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kSBufs; ++i) {
             mbar_init(sf0 + 8 * i, 1);
             mbar_init(pf0 + 8 * i, 128);
-            mbar_init(od0 + 8 * i, 1);
+            mbar_init(sx0 + 8 * i, 1);
         }
         mbar_init(qf, 1);
         mbar_init(qe, 1);
@@ -300,7 +355,7 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const uint32_t tmem = s_tmem;
     pdl_trigger();
 
-    if (warp == 4) {
+    if (warp == kProducerWarp) {
         // ------------------------------------------------ producer (lane 0 issues, the warp resolves rows)
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQ)) : "memory");
@@ -341,18 +396,15 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                             }
                         }
                         if (!dead && !mbar_wait(ke0 + 8 * st, ((uint32_t)(i / kStages) & 1u) ^ 1u, err)) dead = true;
-                        if (!dead) {
-                            mbar_arrive_expect_tx(kf0 + 8 * st, kOperand);
-                            mbar_arrive_expect_tx(vf0 + 8 * st, kOperand);
-                        }
+                        if (!dead) mbar_arrive_expect_tx(kf0 + 8 * st, kStage);
                     }
                     if (!dead) {
                         const uint32_t kd = sKV + (uint32_t)st * kStage + (uint32_t)j * lp.boxh * 128;
                         const uint32_t vd = kd + kOperand;
                         la_tma3(kd, &tmK, 0, cur.h, rq, kf0 + 8 * st, pol);
                         la_tma3(kd + kHalf, &tmK, 64, cur.h, rq, kf0 + 8 * st, pol);
-                        la_tma3(vd, &tmV, 0, cur.h, rq, vf0 + 8 * st, pol);
-                        la_tma3(vd + kHalf, &tmV, 64, cur.h, rq, vf0 + 8 * st, pol);
+                        la_tma3(vd, &tmV, 0, cur.h, rq, kf0 + 8 * st, pol);
+                        la_tma3(vd + kHalf, &tmV, 64, cur.h, rq, kf0 + 8 * st, pol);
                         if (j == lp.nbox - 1) {
                             ++issued;
                             la_next(cur, tab, lp);
@@ -370,69 +422,91 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             for (int64_t i = issued > kStages ? issued - kStages : 0; i < issued; ++i) {
                 const uint32_t par = (uint32_t)(i / kStages) & 1u;
                 mbar_wait(kf0 + 8 * (uint32_t)(i % kStages), par, err);
-                mbar_wait(vf0 + 8 * (uint32_t)(i % kStages), par, err);
             }
             if (qloads > 0) mbar_wait(qf, (uint32_t)(qloads - 1) & 1u, err);
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer (one thread)
+        // Event loop: O(i) goes out as soon as P(i) is in, S(j) as soon as tile j has landed and
+        // S buffer j % kSBufs is free (O(j - kSBufs), which reads the P there, has been issued:
+        // the tcgen05 MMAs of one thread execute in issue order). No product waits behind a
+        // later tile's load, and the loop polls two barriers per tile (each poll of shared
+        // memory is slow while TMA and the tensor core stream through it). No tcgen05 fence
+        // here: in this thread it would wait for the products in flight. The operands are
+        // ordered by the mbarriers: TMA completion for K/V, and tcgen05.wait::st before every
+        // arrival that hands over TMEM written by the softmax threads (P, a rescaled O).
         if (lane == 0) {
             const uint32_t idS = la_idesc(kRows, kTile, false), idO = la_idesc(kRows, kDh, true);
             LaCursor cs = la_cursor(s0, tab, lp), co = cs;
             int qwaits = 0;
+            bool q_ready = false;  // the queries of S tile ns's run have landed
+            int64_t ns = 0, no = 0;  // next S tile, next O tile
+            int64_t run0 = 0;        // first local tile of the run the O products are in
             bool dead = false;
-            // S of tile i into TMEM columns (i & 1) * 64
-            auto issue_s = [&](int64_t i, const LaCursor& u) -> bool {
-                if (i == 0 || u.t == 0) {  // a run starts: its queries must have landed
-                    if (!mbar_wait(qf, (uint32_t)qwaits & 1u, err)) return false;
-                    ++qwaits;
-                }
-                const int st = (int)(i % kStages);
-                if (!mbar_wait(kf0 + 8 * st, (uint32_t)(i / kStages) & 1u, err)) return false;
-                la_fence_after();
-                const uint32_t kb = sKV + (uint32_t)st * kStage;
+            uint64_t t_last = global_timer_ns();
+            uint32_t spins = 0;
+            while (no < n && !dead) {
+                bool prog = false;
+                // S buffer ns % kSBufs holds P(ns - kSBufs): S(ns) goes out after O(ns - kSBufs) has
+                // been issued, and the MMAs of one thread execute in issue order
+                if (ns < n && ns < no + kSBufs) {
+                    const bool run_start = ns == 0 || cs.t == 0;
+                    if (run_start && !q_ready && la_test_wait(qf, (uint32_t)qwaits & 1u)) {
+                        q_ready = true;
+                        ++qwaits;
+                    }
+                    const int st = (int)(ns % kStages);
+                    if ((!run_start || q_ready) && la_test_wait(kf0 + 8 * st, (uint32_t)(ns / kStages) & 1u)) {
+                        const uint32_t kb = sKV + (uint32_t)st * kStage;
+                        const uint32_t d = tmem + (uint32_t)(ns % kSBufs) * kTile;
 #pragma unroll
-                for (int kk = 0; kk < kDh / 16; ++kk) {
-                    const uint64_t a = la_desc(sQ + (uint32_t)(kk >> 2) * kQHalf + (uint32_t)(kk & 3) * 32, 16, 1024);
-                    const uint64_t b = la_desc(kb + (uint32_t)(kk >> 2) * kHalf + (uint32_t)(kk & 3) * 32, 16, 1024);
-                    la_mma(tmem + (uint32_t)(i & 1) * kTile, a, b, idS, kk > 0 ? 1u : 0u);
-                }
-                la_commit(sf0 + 8 * (uint32_t)(i & 1));
-                if (i == n - 1 || u.t == u.nt - 1) la_commit(qe);  // the run's last S: Qd may be replaced
-                return true;
-            };
-            if (n > 0 && !issue_s(0, cs)) dead = true;
-            for (int64_t i = 0; i < n && !dead; ++i) {
-                if (*(volatile int*)&s_abort) {
-                    dead = true;
-                    break;
-                }
-                if (i + 1 < n) {
-                    la_next(cs, tab, lp);
-                    if (!issue_s(i + 1, cs)) {
-                        dead = true;
-                        break;
+                        for (int kk = 0; kk < kDh / 16; ++kk) {
+                            const uint64_t a = la_desc(sQ + (uint32_t)(kk >> 2) * kQHalf + (uint32_t)(kk & 3) * 32, 16, 1024);
+                            const uint64_t b = la_desc(kb + (uint32_t)(kk >> 2) * kHalf + (uint32_t)(kk & 3) * 32, 16, 1024);
+                            la_mma(d, a, b, idS, kk > 0 ? 1u : 0u);
+                        }
+                        la_commit(sf0 + 8 * (uint32_t)(ns % kSBufs));
+                        if (ns == n - 1 || cs.t == cs.nt - 1) la_commit(qe);  // the run's last S: Qd may go
+                        q_ready = false;
+                        ++ns;
+                        if (ns < n) la_next(cs, tab, lp);
+                        prog = true;
                     }
                 }
-                const int st = (int)(i % kStages);
-                if (!mbar_wait(pf0 + 8 * (uint32_t)(i & 1), (uint32_t)(i >> 1) & 1u, err) ||
-                    !mbar_wait(vf0 + 8 * st, (uint32_t)(i / kStages) & 1u, err)) {
-                    dead = true;
-                    break;
-                }
-                la_fence_after();
-                const bool first = (i == 0) || co.t == 0;
-                const uint32_t pa = sP + (uint32_t)(i & 1) * kPBytes;
-                const uint32_t vb = sKV + (uint32_t)st * kStage + kOperand;
+                if (no < ns) {
+                    const int st = (int)(no % kStages);
+                    const uint32_t g = (uint32_t)(no & 1);
+                    // V(no) landed with K(no) (one barrier per stage, seen when S(no) went out)
+                    if (la_test_wait(pf0 + 8 * (uint32_t)(no % kSBufs), (uint32_t)(no / kSBufs) & 1u)) {
+                        if (no == 0 || co.t == 0) run0 = no;
+                        const bool first = no - run0 < 2;  // this group's first tile of the run: O afresh
+                        // P(no) sits in the first 32 columns of S buffer no % kSBufs (bf16 pairs)
+                        const uint32_t pa = tmem + (uint32_t)(no % kSBufs) * kTile;
+                        const uint32_t vb = sKV + (uint32_t)st * kStage + kOperand;
 #pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk) {
-                    const uint64_t a = la_desc(pa + (uint32_t)kk * 32, 16, 1024);
-                    const uint64_t b = la_desc(vb + (uint32_t)kk * 2048, kHalf, 1024);
-                    la_mma(tmem + kTmemO, a, b, idO, (!first || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < kTile / 16; ++kk) {
+                            const uint64_t b = la_desc(vb + (uint32_t)kk * 2048, kHalf, 1024);
+                            la_mma_ts(tmem + kTmemO + g * kDh, pa + (uint32_t)kk * 8, b, idO, (!first || kk > 0) ? 1u : 0u);
+                        }
+                        la_commit(ke0 + 8 * st);
+                        la_commit(sx0 + 8 * (uint32_t)(no % kSBufs));
+                        ++no;
+                        la_next(co, tab, lp);
+                        prog = true;
+                    }
                 }
-                la_commit(od0 + 8 * (uint32_t)(i & 1));
-                la_commit(ke0 + 8 * st);
-                la_next(co, tab, lp);
+                if (prog) {
+                    spins = 0;
+                    t_last = 0;
+                } else if ((++spins & 255u) == 0u) {
+                    // bounded: no progress for kWaitLimitNs (or 2^26 polls) gives up
+                    const uint64_t now = global_timer_ns();
+                    if (t_last == 0) t_last = now;
+                    if (*(volatile int*)&s_abort || now - t_last > kWaitLimitNs || spins >= (1u << 26)) {
+                        if (!*(volatile int*)&s_abort) set_error(err, kErrTimeout);
+                        dead = true;
+                    }
+                }
             }
             if (dead) s_abort = 1;
             // every MMA issued has completed before TMEM is released
@@ -440,165 +514,200 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             mbar_wait(endb, 0, err);
         }
     } else {
-        // ------------------------------------------------ softmax: thread r owns TMEM lane r
-        const int r = tid, half = r >> 6, qrow = r & 63;
-        const uint32_t lane_t = tmem + ((uint32_t)(warp * 32) << 16);
-        const uint32_t prow = (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128;
-        float* scratch = reinterpret_cast<float*>(la_raw + (sP - raw));  // both P tiles, at run ends
+        // ------------------------------------------------ softmax: two groups of 128 threads take
+        // alternate tiles; thread r of a group owns TMEM lane r and its group's O row r
+        const int g = warp >> 2, r = tid & 127, half = r >> 6, qrow = r & 63;
+        const uint32_t lane_t = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const uint32_t o0 = lane_t + kTmemO, o1 = o0 + kDh, o_mine = g ? o1 : o0;
+        float* scratch = reinterpret_cast<float*>(la_raw + (sX - raw));  // run-end merge scratch
         LaCursor cur = la_cursor(s0, tab, lp);
         float m = -INFINITY, l = 0.f;
         bool dead = false, run_whole = false;
         int run_idx = 0;
+        int64_t run0 = 0;
         for (int64_t i = 0; i < n; ++i) {
-            const bool first = (i == 0) || cur.t == 0;
             const bool last = (i == n - 1) || cur.t == cur.nt - 1;
-            if (first) {
+            if (i == 0 || cur.t == 0) {
                 m = -INFINITY;
                 l = 0.f;
                 run_whole = cur.t == 0;
+                run0 = i;
             }
-            // 1. this row's 32 scores of tile i
-            dead = la_wait_warp(dead, sf0 + 8 * (uint32_t)(i & 1), (uint32_t)(i >> 1) & 1u, err, &s_abort);
-            la_fence_after();
-            uint32_t sr[32];
-            if (!dead) {
-                la_ld32(lane_t + (uint32_t)(i & 1) * kTile + (uint32_t)half * 32, sr);
-                la_wait_ld();
-            } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) sr[j] = 0u;
-            }
-            const int rem = cur.kt - (cur.t * kTile + half * 32);
-            const int nvalid = rem < 0 ? 0 : (rem > 32 ? 32 : rem);
-            float x[32], mt = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                x[j] = j < nvalid ? __uint_as_float(sr[j]) * lp.qscale : -INFINITY;
-                mt = fmaxf(mt, x[j]);
-            }
-            // 2. running max; O is rescaled only when the max grows past the threshold
-            const float mn = fmaxf(m, mt);
-            float alpha = 1.f;
-            bool need = false;
-            if (first) {
-                m = mn;
-            } else if (mn > m + kRescale) {
-                need = true;
-                alpha = la_ex2(m - mn);
-                m = mn;
-            }
-            if (__any_sync(0xffffffffu, need)) {
-                dead = la_wait_warp(dead, od0 + 8 * (uint32_t)((i - 1) & 1), (uint32_t)((i - 1) >> 1) & 1u, err,
+            if ((int)(i & 1) == g) {
+                // 1. this row's 32 scores of tile i
+                dead = la_wait_warp(dead, sf0 + 8 * (uint32_t)(i % kSBufs), (uint32_t)(i / kSBufs) & 1u, err,
                                     &s_abort);
                 la_fence_after();
+                uint32_t sr[32];
                 if (!dead) {
+                    la_ld32(lane_t + (uint32_t)(i % kSBufs) * kTile + (uint32_t)half * 32, sr);
+                    la_wait_ld();
+                } else {
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        uint32_t o[32];
-                        la_ld32(lane_t + kTmemO + (uint32_t)cc * 32, o);
-                        la_wait_ld();
+                    for (int j = 0; j < 32; ++j) sr[j] = 0u;
+                }
+                float s[32];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                        la_st32(lane_t + kTmemO + (uint32_t)cc * 32, o);
+                for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(sr[j]);
+                const int rem = cur.kt - (cur.t * kTile + half * 32);
+                if (rem < 32) {  // a ragged last tile: tokens past the kept ones do not count
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (j >= rem) s[j] = -INFINITY;
+                }
+                float mx[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) mx[j] = fmaxf(fmaxf(s[4 * j], s[4 * j + 1]), fmaxf(s[4 * j + 2], s[4 * j + 3]));
+                const float mt =
+                    fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+                    lp.qscale;
+                // 2. running max (log2 domain); O is rescaled only when the max grows past 2^8
+                const float mn = fmaxf(m, mt);
+                float alpha = 1.f;
+                bool need = false;
+                if (i - run0 < 2) {
+                    m = mn;  // this group's first tile of the run: O starts afresh
+                } else if (mn > m + kRescale) {
+                    need = true;
+                    alpha = la_ex2(m - mn);
+                    m = mn;
+                }
+                if (__any_sync(0xffffffffu, need)) {
+                    // the group's previous O product (tile i - 2) has finished: its O row is stable.
+                    // (Waited on the per-buffer barrier: S(i) has landed, so O(i - 4) is done and the
+                    // phase awaited is the pending one or the last completed, never two ahead.)
+                    dead = la_wait_warp(dead, sx0 + 8 * (uint32_t)((i - 2) % kSBufs), (uint32_t)((i - 2) / kSBufs) & 1u,
+                                        err, &s_abort);
+                    la_fence_after();
+                    if (!dead) {
+#pragma unroll 1
+                        for (int cc = 0; cc < kDh / 16; ++cc) {
+                            uint32_t o[16];
+                            la_ld16(o_mine + (uint32_t)cc * 16, o);
+                            la_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                            la_st16(o_mine + (uint32_t)cc * 16, o);
+                        }
+                        la_wait_st();
                     }
+                    l *= alpha;
+                }
+                // 3. P = 2^(s*c - m) in bf16 pairs over the first 32 columns of this S buffer (its
+                // scores are in registers): the 64 tokens of the row, this half's 32 real and the
+                // other half's zero. l sums the fp32 weights.
+                const float nm = m == -INFINITY ? 0.f : -m;  // all masked so far: every p is 2^-inf = 0
+                uint32_t pk[32];
+                float ps[4];
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    float p[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) p[e] = la_ex2(fmaf(s[8 * q8 + e], lp.qscale, nm));
+                    ps[q8] = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(p[2 * e], p[2 * e + 1]);
+                        const uint32_t w = *reinterpret_cast<const uint32_t*>(&h2);
+                        pk[q8 * 4 + e] = half ? 0u : w;
+                        pk[16 + q8 * 4 + e] = half ? w : 0u;
+                    }
+                }
+                l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+                if (!dead) {
+                    la_st32(lane_t + (uint32_t)(i % kSBufs) * kTile, pk);
                     la_wait_st();
                 }
-                l *= alpha;
+                la_fence_before();
+                mbar_arrive(pf0 + 8 * (uint32_t)(i % kSBufs));
             }
-            // 3. P of tile i into P tile (i & 1), free once O(i - 2) has completed
-            if (i >= 2)
-                dead = la_wait_warp(dead, od0 + 8 * (uint32_t)(i & 1), (uint32_t)((i - 2) >> 1) & 1u, err, &s_abort);
-            uint32_t pk[16];
-            float ps = 0.f;
-            const bool live = m != -INFINITY;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float p0 = live ? la_ex2(x[2 * j] - m) : 0.f;
-                const float p1 = live ? la_ex2(x[2 * j + 1] - m) : 0.f;
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                pk[j] = *reinterpret_cast<const uint32_t*>(&h2);
-                ps += bf16lo(pk[j]) + bf16hi(pk[j]);
-            }
-            l += ps;
-            const uint32_t pb = sP + (uint32_t)(i & 1) * kPBytes + prow;
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if ((cc >> 2) == half) {
-                    const int b4 = (cc & 3) * 4;
-                    v = make_uint4(pk[b4], pk[b4 + 1], pk[b4 + 2], pk[b4 + 3]);
-                }
-                la_sts128(pb + ((uint32_t)(cc ^ (r & 7)) << 4), v);
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            la_fence_before();
-            mbar_arrive(pf0 + 8 * (uint32_t)(i & 1));
 
-            // 4. end of this CTA's part of run (b, h): merge the half-rows, write out or a partial
+            // 4. end of this CTA's part of run (b, h): merge the two groups and the two half-rows,
+            // then write out (whole run) or a partial (run split across CTAs)
             if (last) {
-                dead = la_wait_warp(dead, od0 + 8 * (uint32_t)(i & 1), (uint32_t)(i >> 1) & 1u, err, &s_abort);
+                const int64_t jl = ((int)(i & 1) == g) ? i : i - 1;  // this group's last tile of the run
+                if (jl >= run0)
+                    dead = la_wait_warp(dead, sx0 + 8 * (uint32_t)(jl % kSBufs), (uint32_t)(jl / kSBufs) & 1u, err,
+                                        &s_abort);
                 la_fence_after();
-                const bool whole = run_whole && cur.t == cur.nt - 1;
-                if (half == 1) {
-                    s_ml[qrow] = make_float2(m, l);
+                if (g == 1) s_ml1[r] = make_float2(m, l);
+                la_softmax_sync();
+                float M = m, L = l, w0 = 0.f, w1 = 0.f;
+                if (g == 0) {
+                    const float2 b1 = s_ml1[r];
+                    M = fmaxf(m, b1.x);
+                    w0 = m == -INFINITY ? 0.f : la_ex2(m - M);
+                    w1 = b1.x == -INFINITY ? 0.f : la_ex2(b1.x - M);
+                    L = w0 * l + w1 * b1.y;
+                    if (half == 1) {  // rows 64..127: both groups' O rows into the scratch
+                        s_mlh[qrow] = make_float2(M, L);
+#pragma unroll 1
+                        for (int cc = 0; cc < kDh / 16; ++cc) {
+                            uint32_t a[16], bq[16];
+                            if (!dead) {
+                                la_ld16(o0 + (uint32_t)cc * 16, a);
+                                la_ld16(o1 + (uint32_t)cc * 16, bq);
+                                la_wait_ld();
+                            }
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        uint32_t o[32];
-                        if (!dead) {
-                            la_ld32(lane_t + kTmemO + (uint32_t)cc * 32, o);
-                            la_wait_ld();
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) o[j] = 0u;
+                            for (int j = 0; j < 16; ++j) {
+                                float v = 0.f;
+                                if (!dead) {
+                                    v = w0 != 0.f ? w0 * __uint_as_float(a[j]) : 0.f;
+                                    if (w1 != 0.f) v = fmaf(w1, __uint_as_float(bq[j]), v);
+                                }
+                                scratch[(cc * 16 + j) * kQmax + qrow] = v;
+                            }
                         }
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) scratch[(cc * 32 + j) * kQmax + qrow] = __uint_as_float(o[j]);
                     }
                 }
                 la_softmax_sync();
-                if (half == 0) {
-                    const float2 o2 = s_ml[qrow];
-                    const float M = fmaxf(m, o2.x);
-                    const float wa = m == -INFINITY ? 0.f : la_ex2(m - M);
-                    const float wb = o2.x == -INFINITY ? 0.f : la_ex2(o2.x - M);
-                    const float L = wa * l + wb * o2.y;
+                if (g == 0 && half == 0) {
+                    const float2 hb = s_mlh[qrow];
+                    const float M2 = fmaxf(M, hb.x);
+                    const float wa = M == -INFINITY ? 0.f : la_ex2(M - M2);
+                    const float wb = hb.x == -INFINITY ? 0.f : la_ex2(hb.x - M2);
+                    const float L2 = wa * L + wb * hb.y;
+                    const float f0 = wa * w0, f1 = wa * w1;
+                    const bool whole = run_whole && cur.t == cur.nt - 1;
                     const bool wr = qrow < lp.Qw && !dead;
                     const int64_t slot = 2 * (int64_t)c + (run_idx == 0 ? 0 : 1);
                     float* dst = whole ? out + (((int64_t)cur.b * lp.Qw + qrow) * lp.H + cur.h) * kDh
                                        : part_o + (slot * lp.Qw + qrow) * kDh;
-                    const float inv = whole ? 1.f / L : 1.f;
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        uint32_t o[32];
+                    const float inv = whole ? 1.f / L2 : 1.f;
+#pragma unroll 1
+                    for (int cc = 0; cc < kDh / 16; ++cc) {
+                        uint32_t a[16], bq[16];
                         if (!dead) {
-                            la_ld32(lane_t + kTmemO + (uint32_t)cc * 32, o);
+                            la_ld16(o0 + (uint32_t)cc * 16, a);
+                            la_ld16(o1 + (uint32_t)cc * 16, bq);
                             la_wait_ld();
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) o[j] = 0u;
                         }
                         if (wr) {
 #pragma unroll
-                            for (int j = 0; j < 32; j += 4) {
-                                float4 v;
-                                v.x = (wa * __uint_as_float(o[j]) + wb * scratch[(cc * 32 + j) * kQmax + qrow]) * inv;
-                                v.y = (wa * __uint_as_float(o[j + 1]) + wb * scratch[(cc * 32 + j + 1) * kQmax + qrow]) * inv;
-                                v.z = (wa * __uint_as_float(o[j + 2]) + wb * scratch[(cc * 32 + j + 2) * kQmax + qrow]) * inv;
-                                v.w = (wa * __uint_as_float(o[j + 3]) + wb * scratch[(cc * 32 + j + 3) * kQmax + qrow]) * inv;
-                                *reinterpret_cast<float4*>(dst + cc * 32 + j) = v;
+                            for (int j = 0; j < 16; j += 4) {
+                                float v[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    float x = wb != 0.f ? wb * scratch[(cc * 16 + j + e) * kQmax + qrow] : 0.f;
+                                    if (f0 != 0.f) x = fmaf(f0, __uint_as_float(a[j + e]), x);
+                                    if (f1 != 0.f) x = fmaf(f1, __uint_as_float(bq[j + e]), x);
+                                    v[e] = x * inv;
+                                }
+                                *reinterpret_cast<float4*>(dst + cc * 16 + j) = make_float4(v[0], v[1], v[2], v[3]);
                             }
                         }
                     }
                     if (wr) {
                         if (whole) {
                             if (lse != nullptr)
-                                lse[((int64_t)cur.b * lp.Qw + qrow) * lp.H + cur.h] = (M + log2f(L)) * kLn2;
+                                lse[((int64_t)cur.b * lp.Qw + qrow) * lp.H + cur.h] = (M2 + log2f(L2)) * kLn2;
                         } else {
-                            *reinterpret_cast<float2*>(part_ml + (slot * lp.Qw + qrow) * 2) = make_float2(M, L);
+                            *reinterpret_cast<float2*>(part_ml + (slot * lp.Qw + qrow) * 2) = make_float2(M2, L2);
                         }
                     }
                 }
-                la_softmax_sync();  // the scratch is read before the next P tile is written
+                la_softmax_sync();  // the scratch is read before the next P tiles are written
                 ++run_idx;
             }
             la_next(cur, tab, lp);

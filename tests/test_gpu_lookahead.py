@@ -2,10 +2,10 @@
 of the fused lookahead step, against the float64 oracle on the same seeded inputs.
 
 Tolerance (bf16 K/V, 2e-2 absolute on the output, as for the single-query path): the kernel
-rounds each softmax weight p to bf16 (relative error <= 2^-9) and normalises by the sum of the
-rounded weights, so the output is a convex combination whose weights are off by at most
-2 * 2^-9 relative. That bounds the error by 2^-8 * max|V| (~0.018 for these N(0,1) caches), and
-the lse by log(1 + 2^-9) < 2e-3 (4e-3 is checked to leave room for the fp32 score rounding)."""
+rounds each softmax weight p to bf16 for the P.V product (relative error <= 2^-9) and divides
+by the fp32 sum of the unrounded weights, so the output is off by at most
+2^-9 * sum_t p_t |V_t| / sum_t p_t <= 2^-9 * max|V| (~0.009 for these N(0,1) caches). The lse
+comes from fp32 scores and fp32 sums only: 1e-4 absolute."""
 import math
 
 import numpy as np
@@ -19,7 +19,7 @@ from tests import _gpu as G
 pytestmark = pytest.mark.gpu
 
 OUT_ATOL = 2e-2
-LSE_ATOL = 4e-3
+LSE_ATOL = 1e-4
 
 
 @pytest.fixture(scope="module")
