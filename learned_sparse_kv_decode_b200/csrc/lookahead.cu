@@ -13,30 +13,32 @@
 // beyond what the CUDA cores sustain at HBM speed, so both products run as tcgen05 MMAs.
 //
 // One CTA per SM, persistent over a balanced run of tiles:
-//  * A tile is 64 consecutive kept tokens of one (sequence, head). The tiles of all (b, h)
+//  * A tile is 128 consecutive kept tokens of one (sequence, head). The tiles of all (b, h)
 //    form one global list; CTA c takes tiles [c*S/G, (c+1)*S/G) (split-K over the list).
 //  * Warp 8 (producer) streams each tile's K and V rows from the full cache, through the
-//    kept chunk ids (or from a compact resident buffer), with 3-D TMA tile loads into a
-//    5-deep ring in the 128-byte-swizzled layout the MMAs read. No multicast; L2 evict-first.
+//    kept chunk ids (or from a compact resident buffer), with 3-D TMA tile loads in the
+//    128-byte-swizzled layout the MMAs read: a 2-deep K ring (a K tile is free once its S
+//    has completed) and a 3-deep V ring (free once its O has). No multicast; L2 evict-first.
 //  * Warp 9 (one thread) issues the MMAs as their inputs arrive (polling, never blocking on
 //    one barrier while another product is ready):
-//      S  = Qd . K^T   M = 128, N = 64,  K = 128  bf16 -> fp32 TMEM, 4 buffers
-//      O += P . V      M = 128, N = 128, K = 64   P read from TMEM, V an MN-major smem operand
-//    Qd holds the window's queries twice (rows 0-63 and 64-127). Rows 0-63 use the scores
-//    of the tile's tokens 0-31 and rows 64-127 those of tokens 32-63 (their P is zero over
-//    the other half). So each softmax thread owns one (query, half-tile) row, and all four
-//    TMEM lane quarters do work. The MMAs do twice the useful flops; at 128 flop per K/V
-//    byte that still sits well under the tensor-pipe roofline.
+//      S  = Qd . K^T   M = 128, N = 128, K = 128  bf16 -> fp32 TMEM, 2 buffers
+//      O += P . V      M = 128, N = 128, K = 128  P read from TMEM, V an MN-major smem operand
+//    (A K=16 MMA with N <= 128 costs about the same whatever N, so the tile is as wide as
+//    the S product allows.) Qd holds the window's queries twice (rows 0-63 and 64-127). Rows
+//    0-63 use the scores of the tile's tokens 0-63 and rows 64-127 those of tokens 64-127
+//    (their P is zero over the other half). So each softmax thread owns one (query,
+//    half-tile) row, and all four TMEM lane quarters do work. The MMAs do twice the useful
+//    flops; at 128 flop per K/V byte that still sits under the tensor-pipe roofline.
 //  * Warps 0-3 and 4-7 are two softmax groups that take alternate tiles. Each group has
 //    its own running max m and sum l per row (log2 domain) and its own O accumulator in
-//    TMEM, so two tiles' softmax overlap. A thread reads its 32 scores (tcgen05.ld) and
-//    writes its bf16 P row over the first 32 columns of the same S buffer (tcgen05.st); l
+//    TMEM, so two tiles' softmax overlap. A thread reads its 64 scores (tcgen05.ld) and
+//    writes its bf16 P row over the first 64 columns of the same S buffer (tcgen05.st); l
 //    sums the fp32 weights. It rescales its O row only when m grows by more than 8 (2^8);
 //    a stale max is exact after the final division by l.
 //  * Per S buffer, three mbarriers order the hand-offs: S landed, P written, and the O
-//    product that read P completed (the buffer is free for S four tiles later). Each
-//    completes one phase every four tiles, so no waiter can fall or run two phases out
-//    of step (a parity wait would then pass early).
+//    product that read P completed. Each completes one phase every two tiles, and the
+//    hand-offs keep every waiter within one phase of it (a parity wait two phases out of
+//    step would pass early).
 //  * At the end of a (b, h) run, group 0 merges its own and group 1's O rows straight from
 //    TMEM (same lanes), then the two half-rows of each query (log-sum-exp). A run wholly
 //    inside the CTA writes out/lse directly. A run split across CTAs writes a partial
@@ -54,26 +56,28 @@
 namespace lsa {
 
 namespace la {
-constexpr int kTile = 64;                 // kept tokens per tile
+constexpr int kTile = 128;                // kept tokens per tile
+constexpr int kHalfTok = kTile / 2;       // tokens of a tile each MMA row (query copy) attends to
 constexpr int kRows = 128;                // MMA rows: the window's queries, twice
 constexpr int kQmax = 64;                 // window queries per (sequence, head)
-constexpr int kStages = 5;                // K/V ring depth
-constexpr uint32_t kHalf = kTile * 128;   // a 64-dim half of a K or V tile: 64 rows x 128 B
-constexpr uint32_t kOperand = 2 * kHalf;  // a K or V tile (16 KiB)
-constexpr uint32_t kStage = 2 * kOperand; // K + V (32 KiB)
+constexpr int kKStages = 2;               // K ring depth (a K tile is free once its S has completed)
+constexpr int kVStages = 3;               // V ring depth (a V tile is free once its O has completed)
+constexpr uint32_t kHalf = kTile * 128;   // a 64-dim half of a K or V tile: 128 rows x 128 B (16 KiB)
+constexpr uint32_t kOperand = 2 * kHalf;  // a K or V tile (32 KiB)
+
 constexpr uint32_t kQHalf = kRows * 128;  // a 64-dim half of Qd (16 KiB)
 constexpr uint32_t kQBytes = 2 * kQHalf;  // Qd (32 KiB)
 constexpr uint32_t kScratch = kQmax * 128 * 4;  // run-end merge: 64 rows x 128 fp32 (32 KiB)
-constexpr uint32_t kSmem = kQBytes + kScratch + kStages * kStage + 1024;  // + alignment slack
+constexpr uint32_t kSmem = kQBytes + kScratch + (kKStages + kVStages) * kOperand + 1024;  // + alignment slack
 constexpr int kThreads = 320;             // warps 0-7 softmax (two groups of 4), 8 producer, 9 MMA
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kSBufs = 4;                 // S buffers in TMEM
-constexpr uint32_t kTmemCols = 512;       // S: 4 x 64 columns, then O of group 0 and of group 1
+constexpr int kSBufs = 2;                 // S buffers in TMEM (one per softmax group)
+constexpr uint32_t kTmemCols = 512;       // S: 2 x 128 columns, then O of group 0 and of group 1
 constexpr uint32_t kTmemO = kSBufs * kTile;  // first O column (group 0; group 1 follows)
 constexpr float kRescale = 8.0f;          // lazy-rescale threshold (log2 units)
 constexpr float kLn2 = 0.69314718055994531f;
-static_assert(kQBytes % 1024 == 0 && kScratch % 1024 == 0 && kStage % 1024 == 0, "1 KiB swizzle atoms");
+static_assert(kQBytes % 1024 == 0 && kScratch % 1024 == 0 && kOperand % 1024 == 0, "1 KiB swizzle atoms");
 static_assert(kTmemO + 2 * 128 == kTmemCols, "TMEM: S buffers then two O accumulators");
 
 }  // namespace la
@@ -83,8 +87,8 @@ struct LaParams {
     int32_t Qw;       // window queries (1..64)
     int32_t G;        // CTAs
     int32_t indexed;  // K/V read through chunk ids (1) or from compact resident buffers (0)
-    int32_t boxh;     // token rows per TMA box: min(C, 64)
-    int32_t nbox;     // boxes per tile: 64 / boxh
+    int32_t boxh;     // token rows per TMA box: min(C, 128)
+    int32_t nbox;     // boxes per tile: 128 / boxh
     int64_t S;        // tiles in the global list
     float qscale;     // log2(e) / sqrt(Dh)
     int32_t tile_off[kMaxB + 1];  // first tile of each sequence (its H runs follow in head order)
@@ -307,7 +311,8 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           const LaParams lp, uint32_t* err) {
     using namespace la;
     extern __shared__ uint8_t la_raw[];
-    __shared__ __align__(8) uint64_t bar_kvf[kStages], bar_ke[kStages];  // ring stage full / empty
+    __shared__ __align__(8) uint64_t bar_kf[kKStages], bar_ke[kKStages];  // K ring full / empty
+    __shared__ __align__(8) uint64_t bar_vf[kVStages], bar_ve[kVStages];  // V ring full / empty
     // per S buffer b: sf = S landed, pf = P written, sx = the O product reading that P has completed
     __shared__ __align__(8) uint64_t bar_sf[kSBufs], bar_pf[kSBufs], bar_sx[kSBufs];
     __shared__ __align__(8) uint64_t bar_qf, bar_qe, bar_end;
@@ -319,18 +324,22 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x;
     const int64_t s0 = (int64_t)c * lp.S / lp.G, s1 = (int64_t)(c + 1) * lp.S / lp.G;
-    const int64_t n = s1 - s0;
+    const int n = (int)(s1 - s0);  // tiles of this CTA (the list is below 2^31 tiles)
     const uint32_t raw = smem_u32(la_raw);
     const uint32_t sQ = (raw + 1023u) & ~1023u;
-    const uint32_t sX = sQ + kQBytes, sKV = sX + kScratch;
-    const uint32_t kf0 = smem_u32(bar_kvf), ke0 = smem_u32(bar_ke);
+    const uint32_t sX = sQ + kQBytes, sK = sX + kScratch, sV = sK + kKStages * kOperand;
+    const uint32_t kf0 = smem_u32(bar_kf), ke0 = smem_u32(bar_ke), vf0 = smem_u32(bar_vf), ve0 = smem_u32(bar_ve);
     const uint32_t sf0 = smem_u32(bar_sf), pf0 = smem_u32(bar_pf), sx0 = smem_u32(bar_sx);
     const uint32_t qf = smem_u32(&bar_qf), qe = smem_u32(&bar_qe), endb = smem_u32(&bar_end);
 
     if (tid == 0) {
-        for (int i = 0; i < kStages; ++i) {
+        for (int i = 0; i < kKStages; ++i) {
             mbar_init(kf0 + 8 * i, 1);
             mbar_init(ke0 + 8 * i, 1);
+        }
+        for (int i = 0; i < kVStages; ++i) {
+            mbar_init(vf0 + 8 * i, 1);
+            mbar_init(ve0 + 8 * i, 1);
         }
         for (int i = 0; i < kSBufs; ++i) {
             mbar_init(sf0 + 8 * i, 1);
@@ -381,7 +390,7 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (lane == 0 && !dead) {
                     const int64_t i = (p0 + qq) / lp.nbox;
                     const int j = (int)((p0 + qq) % lp.nbox);
-                    const int st = (int)(i % kStages);
+                    const int sk = (int)(i % kKStages), sv = (int)(i % kVStages);
                     if (j == 0) {
                         if (*(volatile int*)&s_abort) dead = true;
                         if (!dead && (i == 0 || cur.t == 0)) {
@@ -395,16 +404,18 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                                 ++qloads;
                             }
                         }
-                        if (!dead && !mbar_wait(ke0 + 8 * st, ((uint32_t)(i / kStages) & 1u) ^ 1u, err)) dead = true;
-                        if (!dead) mbar_arrive_expect_tx(kf0 + 8 * st, kStage);
+                        if (!dead && !mbar_wait(ke0 + 8 * sk, ((uint32_t)(i / kKStages) & 1u) ^ 1u, err)) dead = true;
+                        if (!dead) mbar_arrive_expect_tx(kf0 + 8 * sk, kOperand);
+                        if (!dead && !mbar_wait(ve0 + 8 * sv, ((uint32_t)(i / kVStages) & 1u) ^ 1u, err)) dead = true;
+                        if (!dead) mbar_arrive_expect_tx(vf0 + 8 * sv, kOperand);
                     }
                     if (!dead) {
-                        const uint32_t kd = sKV + (uint32_t)st * kStage + (uint32_t)j * lp.boxh * 128;
-                        const uint32_t vd = kd + kOperand;
-                        la_tma3(kd, &tmK, 0, cur.h, rq, kf0 + 8 * st, pol);
-                        la_tma3(kd + kHalf, &tmK, 64, cur.h, rq, kf0 + 8 * st, pol);
-                        la_tma3(vd, &tmV, 0, cur.h, rq, kf0 + 8 * st, pol);
-                        la_tma3(vd + kHalf, &tmV, 64, cur.h, rq, kf0 + 8 * st, pol);
+                        const uint32_t kd = sK + (uint32_t)sk * kOperand + (uint32_t)j * lp.boxh * 128;
+                        const uint32_t vd = sV + (uint32_t)sv * kOperand + (uint32_t)j * lp.boxh * 128;
+                        la_tma3(kd, &tmK, 0, cur.h, rq, kf0 + 8 * sk, pol);
+                        la_tma3(kd + kHalf, &tmK, 64, cur.h, rq, kf0 + 8 * sk, pol);
+                        la_tma3(vd, &tmV, 0, cur.h, rq, vf0 + 8 * sv, pol);
+                        la_tma3(vd + kHalf, &tmV, 64, cur.h, rq, vf0 + 8 * sv, pol);
                         if (j == lp.nbox - 1) {
                             ++issued;
                             la_next(cur, tab, lp);
@@ -419,10 +430,10 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         }
         if (lane == 0) {
             // the copies still in flight land before the CTA may exit
-            for (int64_t i = issued > kStages ? issued - kStages : 0; i < issued; ++i) {
-                const uint32_t par = (uint32_t)(i / kStages) & 1u;
-                mbar_wait(kf0 + 8 * (uint32_t)(i % kStages), par, err);
-            }
+            for (int64_t i = issued > kKStages ? issued - kKStages : 0; i < issued; ++i)
+                mbar_wait(kf0 + 8 * (uint32_t)(i % kKStages), (uint32_t)(i / kKStages) & 1u, err);
+            for (int64_t i = issued > kVStages ? issued - kVStages : 0; i < issued; ++i)
+                mbar_wait(vf0 + 8 * (uint32_t)(i % kVStages), (uint32_t)(i / kVStages) & 1u, err);
             if (qloads > 0) mbar_wait(qf, (uint32_t)(qloads - 1) & 1u, err);
         }
     } else if (warp == kMmaWarp) {
@@ -440,8 +451,8 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             LaCursor cs = la_cursor(s0, tab, lp), co = cs;
             int qwaits = 0;
             bool q_ready = false;  // the queries of S tile ns's run have landed
-            int64_t ns = 0, no = 0;  // next S tile, next O tile
-            int64_t run0 = 0;        // first local tile of the run the O products are in
+            int ns = 0, no = 0;  // next S tile, next O tile
+            int run0 = 0;        // first local tile of the run the O products are in
             bool dead = false;
             uint64_t t_last = global_timer_ns();
             uint32_t spins = 0;
@@ -455,9 +466,9 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                         q_ready = true;
                         ++qwaits;
                     }
-                    const int st = (int)(ns % kStages);
-                    if ((!run_start || q_ready) && la_test_wait(kf0 + 8 * st, (uint32_t)(ns / kStages) & 1u)) {
-                        const uint32_t kb = sKV + (uint32_t)st * kStage;
+                    const int sk = ns % kKStages;
+                    if ((!run_start || q_ready) && la_test_wait(kf0 + 8 * sk, (uint32_t)(ns / kKStages) & 1u)) {
+                        const uint32_t kb = sK + (uint32_t)sk * kOperand;
                         const uint32_t d = tmem + (uint32_t)(ns % kSBufs) * kTile;
 #pragma unroll
                         for (int kk = 0; kk < kDh / 16; ++kk) {
@@ -466,6 +477,7 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                             la_mma(d, a, b, idS, kk > 0 ? 1u : 0u);
                         }
                         la_commit(sf0 + 8 * (uint32_t)(ns % kSBufs));
+                        la_commit(ke0 + 8 * sk);  // K tile free once this S has completed
                         if (ns == n - 1 || cs.t == cs.nt - 1) la_commit(qe);  // the run's last S: Qd may go
                         q_ready = false;
                         ++ns;
@@ -474,21 +486,21 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     }
                 }
                 if (no < ns) {
-                    const int st = (int)(no % kStages);
+                    const int sv = no % kVStages;
                     const uint32_t g = (uint32_t)(no & 1);
-                    // V(no) landed with K(no) (one barrier per stage, seen when S(no) went out)
-                    if (la_test_wait(pf0 + 8 * (uint32_t)(no % kSBufs), (uint32_t)(no / kSBufs) & 1u)) {
+                    if (la_test_wait(pf0 + 8 * (uint32_t)(no % kSBufs), (uint32_t)(no / kSBufs) & 1u) &&
+                        la_test_wait(vf0 + 8 * sv, (uint32_t)(no / kVStages) & 1u)) {
                         if (no == 0 || co.t == 0) run0 = no;
                         const bool first = no - run0 < 2;  // this group's first tile of the run: O afresh
-                        // P(no) sits in the first 32 columns of S buffer no % kSBufs (bf16 pairs)
+                        // P(no) sits in the first 64 columns of S buffer no % kSBufs (bf16 pairs)
                         const uint32_t pa = tmem + (uint32_t)(no % kSBufs) * kTile;
-                        const uint32_t vb = sKV + (uint32_t)st * kStage + kOperand;
+                        const uint32_t vb = sV + (uint32_t)sv * kOperand;
 #pragma unroll
                         for (int kk = 0; kk < kTile / 16; ++kk) {
                             const uint64_t b = la_desc(vb + (uint32_t)kk * 2048, kHalf, 1024);
                             la_mma_ts(tmem + kTmemO + g * kDh, pa + (uint32_t)kk * 8, b, idO, (!first || kk > 0) ? 1u : 0u);
                         }
-                        la_commit(ke0 + 8 * st);
+                        la_commit(ve0 + 8 * sv);  // V tile free once this O has completed
                         la_commit(sx0 + 8 * (uint32_t)(no % kSBufs));
                         ++no;
                         la_next(co, tab, lp);
@@ -524,8 +536,8 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         float m = -INFINITY, l = 0.f;
         bool dead = false, run_whole = false;
         int run_idx = 0;
-        int64_t run0 = 0;
-        for (int64_t i = 0; i < n; ++i) {
+        int run0 = 0;
+        for (int i = 0; i < n; ++i) {
             const bool last = (i == n - 1) || cur.t == cur.nt - 1;
             if (i == 0 || cur.t == 0) {
                 m = -INFINITY;
@@ -538,29 +550,33 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 dead = la_wait_warp(dead, sf0 + 8 * (uint32_t)(i % kSBufs), (uint32_t)(i / kSBufs) & 1u, err,
                                     &s_abort);
                 la_fence_after();
-                uint32_t sr[32];
-                if (!dead) {
-                    la_ld32(lane_t + (uint32_t)(i % kSBufs) * kTile + (uint32_t)half * 32, sr);
-                    la_wait_ld();
-                } else {
+                // this row's 64 scores (tokens half*64 .. half*64+63 of the tile) are read twice from
+                // TMEM, 32 at a time: once for the tile max, once for P (fewer live registers)
+                const uint32_t sbuf = lane_t + (uint32_t)(i % kSBufs) * kTile;
+                const int rem = cur.kt - (cur.t * kTile + half * kHalfTok);  // valid tokens of the row
+                float mt = -INFINITY;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) sr[j] = 0u;
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t sr[32];
+                    if (!dead) {
+                        la_ld32(sbuf + (uint32_t)(half * kHalfTok + hh * 32), sr);
+                        la_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) sr[j] = 0u;
+                    }
+                    float mx[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        float v[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            v[e] = hh * 32 + 8 * j + e < rem ? __uint_as_float(sr[8 * j + e]) : -INFINITY;
+                        mx[j] = fmaxf(fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])), fmaxf(fmaxf(v[4], v[5]), fmaxf(v[6], v[7])));
+                    }
+                    mt = fmaxf(mt, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
                 }
-                float s[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(sr[j]);
-                const int rem = cur.kt - (cur.t * kTile + half * 32);
-                if (rem < 32) {  // a ragged last tile: tokens past the kept ones do not count
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (j >= rem) s[j] = -INFINITY;
-                }
-                float mx[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) mx[j] = fmaxf(fmaxf(s[4 * j], s[4 * j + 1]), fmaxf(s[4 * j + 2], s[4 * j + 3]));
-                const float mt =
-                    fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
-                    lp.qscale;
+                mt *= lp.qscale;
                 // 2. running max (log2 domain); O is rescaled only when the max grows past 2^8
                 const float mn = fmaxf(m, mt);
                 float alpha = 1.f;
@@ -593,29 +609,47 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     }
                     l *= alpha;
                 }
-                // 3. P = 2^(s*c - m) in bf16 pairs over the first 32 columns of this S buffer (its
-                // scores are in registers): the 64 tokens of the row, this half's 32 real and the
+                // 3. P = 2^(s*c - m) in bf16 pairs over the first 64 columns of this S buffer (its
+                // scores are in registers): the row's 128 tokens, this half's 64 real and the
                 // other half's zero. l sums the fp32 weights.
                 const float nm = m == -INFINITY ? 0.f : -m;  // all masked so far: every p is 2^-inf = 0
-                uint32_t pk[32];
-                float ps[4];
+                float ps[8];
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    float p[8];
+                for (int hb = 0; hb < 2; ++hb) {  // 32 tokens (16 columns of P) at a time
+                    uint32_t sr[32];
+                    if (!dead) {
+                        la_ld32(sbuf + (uint32_t)(half * kHalfTok + hb * 32), sr);
+                        la_wait_ld();
+                    } else {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) p[e] = la_ex2(fmaf(s[8 * q8 + e], lp.qscale, nm));
-                    ps[q8] = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(p[2 * e], p[2 * e + 1]);
-                        const uint32_t w = *reinterpret_cast<const uint32_t*>(&h2);
-                        pk[q8 * 4 + e] = half ? 0u : w;
-                        pk[16 + q8 * 4 + e] = half ? w : 0u;
+                        for (int j = 0; j < 32; ++j) sr[j] = 0u;
                     }
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8) {
+                        float p[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int j = hb * 32 + 8 * q8 + e;
+                            p[e] = j < rem ? la_ex2(fmaf(__uint_as_float(sr[8 * q8 + e]), lp.qscale, nm)) : 0.f;
+                        }
+                        ps[hb * 4 + q8] = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const __nv_bfloat162 h2 = __floats2bfloat162_rn(p[2 * e], p[2 * e + 1]);
+                            pk[q8 * 4 + e] = *reinterpret_cast<const uint32_t*>(&h2);
+                        }
+                    }
+                    // P columns half*32 + hb*16 .. +15 hold scores this row has already read
+                    if (!dead) la_st16(sbuf + (uint32_t)(half * 32 + hb * 16), pk);
                 }
-                l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+                l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
                 if (!dead) {
-                    la_st32(lane_t + (uint32_t)(i % kSBufs) * kTile, pk);
+                    uint32_t zero[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) zero[j] = 0u;
+                    la_st16(sbuf + (uint32_t)((1 - half) * 32), zero);
+                    la_st16(sbuf + (uint32_t)((1 - half) * 32 + 16), zero);
                     la_wait_st();
                 }
                 la_fence_before();
@@ -625,7 +659,7 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             // 4. end of this CTA's part of run (b, h): merge the two groups and the two half-rows,
             // then write out (whole run) or a partial (run split across CTAs)
             if (last) {
-                const int64_t jl = ((int)(i & 1) == g) ? i : i - 1;  // this group's last tile of the run
+                const int jl = ((i & 1) == g) ? i : i - 1;  // this group's last tile of the run
                 if (jl >= run0)
                     dead = la_wait_warp(dead, sx0 + 8 * (uint32_t)(jl % kSBufs), (uint32_t)(jl / kSBufs) & 1u, err,
                                         &s_abort);
@@ -731,6 +765,7 @@ k_attn_la_merge(const float* __restrict__ part_o, const float* __restrict__ part
     const int g = blockIdx.x, b = g / lp.H, h = g - b * lp.H;
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = blockIdx.y * 8 + w;
+    pdl_trigger();  // the next kernel may set itself up; its reads wait for this grid
     pdl_wait();
     if (q >= lp.Qw) return;
     const int kt = (tab.kept_off[b + 1] - tab.kept_off[b]) * tab.C;
@@ -748,6 +783,7 @@ k_attn_la_merge(const float* __restrict__ part_o, const float* __restrict__ part
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
     float L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    constexpr int kU = 8;  // partial rows in flight per lane
     for (int i0 = 0; i0 < ns; i0 += 32) {
         float wgt = 0.f;
         if (i0 + lane < ns) {
@@ -756,14 +792,23 @@ k_attn_la_merge(const float* __restrict__ part_o, const float* __restrict__ part
             L = fmaf(wgt, ml.y, L);
         }
         const int cnt = ns - i0 < 32 ? ns - i0 : 32;
-        for (int jj = 0; jj < cnt; ++jj) {
-            const float wj = __shfl_sync(0xffffffffu, wgt, jj);
-            const float4 v = *reinterpret_cast<const float4*>(part_o + ((int64_t)slot_of(i0 + jj) * lp.Qw + q) * kDh +
-                                                              lane * 4);
-            acc.x = fmaf(wj, v.x, acc.x);
-            acc.y = fmaf(wj, v.y, acc.y);
-            acc.z = fmaf(wj, v.z, acc.z);
-            acc.w = fmaf(wj, v.w, acc.w);
+        for (int j0 = 0; j0 < cnt; j0 += kU) {
+            float4 v[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u)
+                v[u] = j0 + u < cnt ? *reinterpret_cast<const float4*>(
+                                          part_o + ((int64_t)slot_of(i0 + j0 + u) * lp.Qw + q) * kDh + lane * 4)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const float wj = __shfl_sync(0xffffffffu, wgt, (j0 + u) & 31);
+                if (j0 + u < cnt) {
+                    acc.x = fmaf(wj, v[u].x, acc.x);
+                    acc.y = fmaf(wj, v[u].y, acc.y);
+                    acc.z = fmaf(wj, v[u].z, acc.z);
+                    acc.w = fmaf(wj, v[u].w, acc.w);
+                }
+            }
         }
     }
     for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);

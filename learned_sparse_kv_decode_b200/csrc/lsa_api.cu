@@ -354,11 +354,13 @@ lsa_status lsa_sparse_decode_attn_lookahead(const lsa_dims* dims, const void* q,
     if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return LSA_ERR_INVALID_ARG;
     if (chunk_ids != nullptr && !aligned16(chunk_ids)) return LSA_ERR_INVALID_ARG;
     if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LSA_ERR_INVALID_ARG;
+    // programmatic dependent launch: every global read of the kernel follows its grid-dependency
+    // wait, so only its prologue (TMEM, barriers) overlaps the previous kernel in the stream
     return cuda_status(launch_attention_la(*dims, p.tab, di.la_ctas, q, K, V, kv_rows, chunk_ids,
                                            reinterpret_cast<float*>(at(ws, w.la_o)),
                                            reinterpret_cast<float*>(at(ws, w.la_ml)), out, lse,
                                            reinterpret_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream),
-                                           false));
+                                           true));
 }
 
 lsa_status lsa_decode_step_lookahead(const lsa_dims* dims, const void* q_emb, const void* chunk_emb, const void* q,
