@@ -44,7 +44,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="128k", choices=["tiny", "128k", "128k-b2", "500k", "1m", "1m-h2", "mixed"])
-    p.add_argument("--contexts", default="500k,1m",
+    p.add_argument("--contexts", default="500k,1m,mixed,tiny",
                    help="extra workloads timed in the same run (comma list, '' for none)")
     p.add_argument("--rotations", type=int, default=4, help="distinct query sets cycled over the steps")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")

@@ -232,6 +232,24 @@ def test_attention_weights_sum_to_one():
     np.testing.assert_allclose(np.exp(z - lse[None, :]).sum(axis=0), 1.0, rtol=0, atol=1e-12)
 
 
+def test_attention_split_merge_is_associative():
+    # attention over a token set split into parts, recombined with the log-sum-exp rule, equals
+    # attention over the whole set (the split-K identity the GPU kernels rely on); this also
+    # pins the lse the oracle returns
+    rng = np.random.default_rng(12)
+    T, H, Dh = 300, 4, 128
+    q, K, V = 2 * rng.standard_normal((H, Dh)), rng.standard_normal((T, H, Dh)), rng.standard_normal((T, H, Dh))
+    out, lse = oracle.attention(q, K, V)
+    for cuts in ([0, 1, 300], [0, 100, 101, 250, 300], [0, 37, 74, 111, 148, 185, 222, 259, 300]):
+        parts = [oracle.attention(q, K[a:b], V[a:b]) for a, b in zip(cuts[:-1], cuts[1:])]
+        M = np.max([l for _, l in parts], axis=0)
+        wts = [np.exp(l - M) for _, l in parts]
+        L = np.sum(wts, axis=0)
+        merged = np.sum([w[:, None] * o for w, (o, _) in zip(wts, parts)], axis=0) / L[:, None]
+        np.testing.assert_allclose(merged, out, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(M + np.log(L), lse, rtol=0, atol=1e-13)
+
+
 def test_attention_scale_is_one_over_sqrt_dh():
     # with scale = 1/sqrt(Dh) by default, doubling Dh-normalised logits must match an explicit scale
     rng = np.random.default_rng(9)
@@ -305,6 +323,21 @@ def test_planted_chunks_recovered_tiny():
     planted = datagen.planted_positions(w, 0)
     assert len(planted) == 4
     assert set(planted.tolist()) <= set(ids.tolist())
+
+
+def test_planted_chunks_recovered_128k():
+    # every sequence of the 128K workload plants 32 chunks near its query embedding; all 32
+    # must be among the 256 kept
+    w = datagen.workload("128k")
+    x = datagen.make_inputs(w)
+    off = w.chunk_offsets
+    for b in range(w.B):
+        s = oracle.chunk_scores(datagen.as_f32(x["q_emb"][b], w.emb_dtype),
+                                datagen.as_f32(x["chunk_emb"][off[b]:off[b + 1]], w.emb_dtype))
+        ids = oracle.topk(s, w.k[b])
+        planted = datagen.planted_positions(w, b)
+        assert len(planted) == 32
+        assert set(planted.tolist()) <= set(ids.tolist())
 
 
 # ---------------------------------------------------------------- resident refresh
