@@ -63,7 +63,7 @@ typedef enum {
     LSA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
     LSA_ERR_NONFINITE = 4,    /* device: a chunk score was NaN or +-Inf */
     LSA_ERR_TIMEOUT = 5,      /* device: a bounded wait gave up */
-    LSA_ERR_UNSUPPORTED = 6,  /* a shape this build does not implement */
+    LSA_ERR_UNSUPPORTED = 6,  /* a shape the library does not implement */
     LSA_ERR_BAD_ID = 7        /* device: a kept chunk id was outside 0..N_b-1 */
 } lsa_status;
 
