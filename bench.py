@@ -185,6 +185,29 @@ def oracle_sample(w, seconds: float = None, steps: int = None, warmup: int = 0):
     return {"t_step": t_step, "items": i - warmup, "sample": sample, "elapsed": time.perf_counter() - t_begin}
 
 
+def _oracle_sample_worker(args):
+    name, seconds = args
+    import datagen
+    return oracle_sample(datagen.workload(name), seconds=seconds, warmup=1)["t_step"]
+
+
+def oracle_sample_all_cores(w, seconds: float) -> dict:
+    """The same oracle sample run in one process per host core (at most 32) at once (spawned workers, so the
+    CUDA context of this process is not forked). The (sequence, head) items of a step are
+    independent, so the step costs the mean single-process step time divided by the process
+    count; measuring them concurrently charges the memory-bandwidth contention."""
+    import multiprocessing as mp
+
+    avail = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    procs = max(1, min(avail, 32))  # each worker prepares its own inputs: bound memory and start-up
+    with mp.get_context("spawn").Pool(procs) as pool:
+        ts = pool.map(_oracle_sample_worker, [(w.name, seconds)] * procs)
+    t_step = sum(ts) / len(ts) / procs
+    return {"value": 1.0 / t_step, "unit": "steps/s", "cores": procs, "kind": "oracle",
+            "sample": f"{procs} concurrent processes, each timing the 1-thread sample for {seconds:.0f} s; "
+                      "step time = mean per-process step time / processes"}
+
+
 def run_reference(args):
     """The reference arm: the float64 oracle on the host cores (rank 0 only)."""
     if int(os.environ.get("RANK", "0")) != 0:
@@ -388,6 +411,17 @@ def run_ours(args):
             res["lookahead"] = lookahead_loop(S, K, W, world, peak)
         if name == args.workload:
             head = S
+            # the distribution of single steps (each replay bracketed by its own events)
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(200)]
+            torch.cuda.synchronize()
+            for i, (e0, e1) in enumerate(ev):
+                e0.record()
+                S.graphs[i % R].replay()
+                e1.record()
+            torch.cuda.synchronize()
+            per = sorted(e0.elapsed_time(e1) * 1e3 for e0, e1 in ev)
+            res["step_us"] = {"p10": per[20], "p50": per[100], "p90": per[180], "n": len(per),
+                              "note": "each replay timed alone (so each includes one graph-launch gap)"}
             # the dominant kernel alone: split-K attention (+ its merge) over the last step's kept ids
             r_last = (K - 1) % R
             ams = time_loop(lambda i: lsa.lsa_sparse_decode_attn(S.dims, S.q[r_last], S.K, S.V, S.ids, S.out,
@@ -416,6 +450,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         r = oracle_sample(w, seconds=args.cpu_seconds, warmup=2)
         cpu = {"value": 1.0 / r["t_step"], "unit": "steps/s", "cores": 1, "kind": "oracle", "sample": r["sample"]}
+        cpu_all = oracle_sample_all_cores(w, args.cpu_seconds)
     if rank == 0:
         e2e = hr["e2e"]
         line = {
@@ -463,6 +498,7 @@ def run_ours(args):
         }
         if cpu is not None:
             line["cpu_baseline"] = cpu
+            line["cpu_baseline_all_cores"] = cpu_all
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
