@@ -212,3 +212,21 @@ def test_lookahead_argument_errors(lsa):
     with pytest.raises(lsa.LsaError) as e:
         lsa.lsa_sparse_decode_attn_lookahead(dw2.dims, q2, dw2.K, dw2.V, dw2.ids, out2, None, dw2.ws)
     assert e.value.status == lsa.LSA_ERR_UNSUPPORTED  # more than 64 window queries
+
+
+def test_lookahead_max_batch_many_runs_per_cta(lsa):
+    # 256 short ragged sequences (C = 16, so ragged last tiles) and 2 heads: 564 tiles over the
+    # CTAs, up to four (sequence, head) runs in one CTA (first split, whole ones, last split)
+    rng = np.random.default_rng(3)
+    N = tuple(int(x) for x in rng.integers(4, 13, size=256))
+    k = tuple(int(rng.integers(1, n + 1)) for n in N)
+    w = datagen.small_workload(B=256, N=N, k=k, E=64, Q=7, H=2, C=16, emb_dtype="bf16", kv_dtype="bf16", seed=66)
+    win = Window(w, lsa)
+    ids = win.random_ids(11)
+    ids_d = torch.from_numpy(np.concatenate(ids)).cuda()
+    lsa.lsa_sparse_decode_attn_lookahead(win.dw.dims, win.q, win.dw.K, win.dw.V, ids_d, win.out, win.lse, win.dw.ws)
+    assert lsa.lsa_get_device_status(win.dw.ws) == lsa.LSA_OK
+    for b in range(w.B):
+        _compare(win, b, ids[b])
+    del win
+    _free()

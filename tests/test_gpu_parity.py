@@ -267,6 +267,19 @@ def test_decode_step_small(lsa, case):
     _check_step(dw)
 
 
+def test_decode_step_max_batch(lsa):
+    # LSA_MAX_BATCH sequences, ragged lengths and keep counts, in one call
+    rng = np.random.default_rng(21)
+    N = tuple(int(x) for x in rng.integers(1, 40, size=256))
+    k = tuple(int(rng.integers(1, n + 1)) for n in N)
+    w = datagen.small_workload(B=256, N=N, k=k, E=64, H=2, C=16, emb_dtype="bf16", kv_dtype="bf16", seed=45)
+    dw = G.DeviceWorkload(w, lsa)
+    _run_step(lsa, dw)
+    _check_step(dw)
+    del dw
+    _free()
+
+
 def test_decode_step_deterministic(lsa):
     w = datagen.small_workload(B=2, N=(300, 129), k=(40, 7), E=128, H=16, emb_dtype="bf16", kv_dtype="bf16")
     dw = G.DeviceWorkload(w, lsa)
