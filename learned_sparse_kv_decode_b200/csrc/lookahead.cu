@@ -227,17 +227,6 @@ __device__ __forceinline__ void la_st16(uint32_t taddr, const uint32_t (&r)[16])
         : "memory");
 }
 
-__device__ __forceinline__ void la_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-        "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
-
 __device__ __forceinline__ void la_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void la_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -259,11 +248,6 @@ __device__ __forceinline__ void la_tma4(uint32_t dst, const CUtensorMap* map, in
         " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
         : "memory");
-}
-
-__device__ __forceinline__ void la_sts128(uint32_t addr, uint4 v) {
-    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                 : "memory");
 }
 
 __device__ __forceinline__ float la_ex2(float x) {
@@ -546,7 +530,7 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 run0 = i;
             }
             if ((int)(i & 1) == g) {
-                // 1. this row's 32 scores of tile i
+                // 1. this row's scores of tile i
                 dead = la_wait_warp(dead, sf0 + 8 * (uint32_t)(i % kSBufs), (uint32_t)(i / kSBufs) & 1u, err,
                                     &s_abort);
                 la_fence_after();
