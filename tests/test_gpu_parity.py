@@ -118,6 +118,24 @@ def test_topk_signed_zero_and_all_equal(lsa):
     np.testing.assert_array_equal(got[11:], [0, 1, 2, 3, 4, 5])
 
 
+@pytest.mark.parametrize("k", [1, 17, 150, 299])
+def test_topk_subnormal_scores(lsa, k):
+    # subnormals of both signs, the smallest normals and +-0, repeated (ties): the
+    # order-preserving key map must order them as floats do, with no flush to zero
+    sub = np.array([1, 2, 3, 7, 1000, 2**22 - 1], np.uint32).view(np.float32)
+    tiny = np.finfo(np.float32).tiny
+    base = np.concatenate([sub, -sub, np.array([tiny, -tiny, 2 * tiny, -3 * tiny, 0.0, -0.0], np.float32)])
+    rng = np.random.default_rng(31)
+    s = rng.permutation(np.tile(base, 25)).astype(np.float32)   # 450 scores
+    w = datagen.small_workload(B=1, N=(len(s),), k=(k,), E=64)
+    dims = G.dims_of(w, lsa)
+    ws = lsa.alloc_workspace(dims)
+    ids = torch.empty(k, dtype=torch.int32, device="cuda")
+    lsa.lsa_topk_select(dims, torch.from_numpy(s).cuda(), ids, ws)
+    assert lsa.lsa_get_device_status(ws) == lsa.LSA_OK
+    np.testing.assert_array_equal(ids.cpu().numpy(), oracle.topk(s.astype(np.float64), k))
+
+
 def test_topk_nonfinite_reported(lsa):
     w = datagen.small_workload(B=1, N=(50,), k=(10,), E=64)
     dims = G.dims_of(w, lsa)
