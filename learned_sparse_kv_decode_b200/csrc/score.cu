@@ -320,6 +320,134 @@ k_score_umma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     }
 }
 
+// Shared-memory descriptor of a K-major operand in the 128-byte-swizzled layout (sm_100 layout
+// type 2): rows of 128 bytes (64 bf16), 8-row atoms of 1 KiB (SBO = 1024); LBO unused (1).
+__device__ __forceinline__ uint64_t umma_desc_k_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// The same GEMM + row max with 128-byte-swizzled operand tiles, for E a multiple of 64 (<= 256).
+// The E dimension is split into E/64 regions of 64 columns; one TMA box per region and operand
+// (box [64 x 128 rows] for the chunks, [64 x Np] for the queries) lands in 128-byte rows, and
+// each region has its own mbarrier so the MMAs of region r start while later regions land.
+// grid (ceil(maxN/128), B), 128 threads; dynamic smem: E/64 * (128 + Np) * 128 B + 1 KiB.
+constexpr int kScoreSwRegionsMax = 4;
+__global__ void __launch_bounds__(128)
+k_score_umma_sw(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                float* __restrict__ scores, const SeqTable tab, int Q, int Np, int E, uint32_t tmem_cols,
+                uint32_t* err) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t load_bar[kScoreSwRegionsMax];
+    __shared__ __align__(8) uint64_t mma_bar;
+    __shared__ uint32_t tmem_slot;
+
+    const int b = blockIdx.y;
+    const int n_b = tab.chunk_off[b + 1] - tab.chunk_off[b];
+    const int r0 = blockIdx.x * kUmmaM;
+    pdl_trigger();
+    if (r0 >= n_b) return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int R = E / 64;  // regions of 64 columns
+    const uint32_t sA = (smem_u32(smem_raw) + 1023u) & ~1023u;  // swizzle atoms need 1 KiB alignment
+    const uint32_t sB = sA + (uint32_t)R * kUmmaM * 128;
+
+    if (tid == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+        for (int r = 0; r < R; ++r) mbar_init(smem_u32(&load_bar[r]), 1);
+        mbar_init(smem_u32(&mma_bar), 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&tmem_slot)),
+                     "r"(tmem_cols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_d = tmem_slot;
+
+    bool loaded = true;
+    if (tid == 0) {
+        // rows past the tensor read as zeros; rows of the next sequence are loaded and masked
+        pdl_wait();
+        const int rowA = tab.chunk_off[b] + r0, rowB = b * Q;
+        for (int r = 0; r < R; ++r) {
+            const uint32_t lb = smem_u32(&load_bar[r]);
+            mbar_arrive_expect_tx(lb, (uint32_t)(kUmmaM + Np) * 128);
+            tma_load_2d(sA + (uint32_t)r * kUmmaM * 128, &tmA, 64 * r, rowA, lb);
+            tma_load_2d(sB + (uint32_t)r * Np * 128, &tmB, 64 * r, rowB, lb);
+        }
+        const uint32_t idesc = umma_idesc_bf16_f32(kUmmaM, Np);
+        for (int r = 0; r < R && loaded; ++r) {
+            loaded = mbar_wait(smem_u32(&load_bar[r]), 0, err);
+            if (!loaded) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {  // 16 columns (32 bytes) per MMA K-step
+                const uint64_t ad = umma_desc_k_sw128(sA + (uint32_t)r * kUmmaM * 128 + (uint32_t)kk * 32);
+                const uint64_t bd = umma_desc_k_sw128(sB + (uint32_t)r * Np * 128 + (uint32_t)kk * 32);
+                const uint32_t accum = (r > 0 || kk > 0) ? 1u : 0u;
+                asm volatile(
+                    "{\n\t.reg .pred p;\n\t"
+                    "setp.ne.b32 p, %4, 0;\n\t"
+                    "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+                    "l"(ad), "l"(bd), "r"(idesc), "r"(accum)
+                    : "memory");
+            }
+        }
+        if (loaded) {
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                             smem_u32(&mma_bar))
+                         : "memory");
+        } else {
+            // a load gave up: wait (bounded) for every copy issued, then release the waiters
+            for (int r = 0; r < R; ++r) mbar_wait(smem_u32(&load_bar[r]), 0, err);
+            mbar_arrive(smem_u32(&mma_bar));
+        }
+    }
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&mma_bar), 0, err) && loaded);
+    const bool all_ok = __syncthreads_and(ok);
+    tc_fence_after();
+
+    // ---- epilogue: row r0 + 32*warp + lane lives in TMEM lane 32*warp + lane
+    float best = -INFINITY;
+    if (all_ok) {
+        const uint32_t taddr = tmem_d + ((uint32_t)(warp * 32) << 16);
+        for (int c0 = 0; c0 < Np; c0 += 16) {
+            uint32_t rr[16];
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                : "=r"(rr[0]), "=r"(rr[1]), "=r"(rr[2]), "=r"(rr[3]), "=r"(rr[4]), "=r"(rr[5]),
+                  "=r"(rr[6]), "=r"(rr[7]), "=r"(rr[8]), "=r"(rr[9]), "=r"(rr[10]), "=r"(rr[11]),
+                  "=r"(rr[12]), "=r"(rr[13]), "=r"(rr[14]), "=r"(rr[15])
+                : "r"(taddr + (uint32_t)c0));
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (c0 + i < Q) best = fmaxf(best, __uint_as_float(rr[i]));
+        }
+        const int row = r0 + warp * 32 + lane;
+        if (row < n_b) scores[tab.chunk_off[b] + row] = best;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d),
+                     "r"(tmem_cols)
+                     : "memory");
+    }
+}
+
+// Host: a 2-D tensor map over a row-major bf16 matrix [rows][cols], box [64 columns x box_rows],
+// 128-byte swizzle, zero fill outside the tensor (cols a multiple of 64).
+cudaError_t make_tmap_sw128(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+
 // Host: a 2-D tensor map over a row-major bf16 matrix [rows][cols] with a box of
 // [box_rows x 8 columns] (16 bytes per row), no swizzle, zero fill outside the tensor.
 cudaError_t make_tmap_rows16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
@@ -342,14 +470,35 @@ cudaError_t make_tmap_rows16(CUtensorMap* map, const void* base, uint64_t rows, 
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t make_tmap_sw128(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (encode == nullptr) {
+        cudaDriverEntryPointQueryResult q;
+        void* fn = nullptr;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr) return cudaErrorInvalidValue;
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // ============================================================== launchers
 // Raise the dynamic shared-memory limit of the score kernels (once per device).
 // The limits are the largest requests the launchers make (E <= 256 and Q <= 256 for the
 // tensor-core kernel; Q*E*4 <= 200 KiB for the stream kernel, checked on the host).
 constexpr int kScoreStreamSmemMax = 200 * 1024;
 size_t score_umma_smem(int E, int Np);
+size_t score_umma_sw_smem(int E, int Np);
 cudaError_t score_init_attrs() {
     cudaError_t e = set_smem_attrs(k_score_umma, (int)score_umma_smem(256, 256));
+    if (e == cudaSuccess) e = set_smem_attrs(k_score_umma_sw, (int)score_umma_sw_smem(256, 256));
     if (e == cudaSuccess) e = set_smem_attrs(k_score_stream<true>, kScoreStreamSmemMax);
     if (e == cudaSuccess) e = set_smem_attrs(k_score_stream<false>, kScoreStreamSmemMax);
     return e;
@@ -357,6 +506,8 @@ cudaError_t score_init_attrs() {
 
 // A and B tiles plus 4 KiB of slack after them (never read when the descriptors are right).
 size_t score_umma_smem(int E, int Np) { return (size_t)(kUmmaM + Np) * E * 2 + 4096; }
+// E/64 regions of (128 + Np) rows x 128 B, plus 1 KiB to align the swizzle atoms.
+size_t score_umma_sw_smem(int E, int Np) { return (size_t)(E / 64) * (kUmmaM + Np) * 128 + 1024; }
 
 bool score_uses_umma(const lsa_dims& d) {
     return d.Q > 1 && d.emb_dtype == LSA_BF16 && d.E % 16 == 0 && d.E <= 256 && d.Q <= 256;
@@ -378,6 +529,15 @@ cudaError_t launch_score(const lsa_dims& d, const SeqTable& tab, int max_n, cons
         uint32_t cols = 32;
         while ((int)cols < Np) cols <<= 1;
         CUtensorMap tmA, tmB;
+        cfg.gridDim = dim3((max_n + kUmmaM - 1) / kUmmaM, d.B, 1);
+        cfg.blockDim = dim3(128, 1, 1);
+        if (d.E % 64 == 0) {  // 128-byte rows: one TMA box per 64-column region and operand
+            cudaError_t e = make_tmap_sw128(&tmA, chunk_emb, (uint64_t)tab.chunk_off[d.B], d.E, kUmmaM);
+            if (e == cudaSuccess) e = make_tmap_sw128(&tmB, q_emb, (uint64_t)d.B * d.Q, d.E, (uint32_t)Np);
+            if (e != cudaSuccess) return e;
+            cfg.dynamicSmemBytes = score_umma_sw_smem(d.E, Np);
+            return cudaLaunchKernelEx(&cfg, k_score_umma_sw, tmA, tmB, scores, tab, d.Q, Np, d.E, cols, err);
+        }
         cudaError_t e = make_tmap_rows16(&tmA, chunk_emb, (uint64_t)tab.chunk_off[d.B], d.E, kUmmaM);
         if (e == cudaSuccess) e = make_tmap_rows16(&tmB, q_emb, (uint64_t)d.B * d.Q, d.E, (uint32_t)Np);
         if (e != cudaSuccess) return e;

@@ -60,6 +60,9 @@ SCORE_CASES = [
     dict(name="umma-Q64-E128", emb_dtype="bf16", E=128, Q=64, N=(513, 7)),
     dict(name="umma-Q3-E64", emb_dtype="bf16", E=64, Q=3, N=(260,)),
     dict(name="umma-Q200-E128", emb_dtype="bf16", E=128, Q=200, N=(140, 120)),
+    dict(name="umma-Q256-E256", emb_dtype="bf16", E=256, Q=256, N=(200, 3)),   # largest swizzled tiles
+    dict(name="umma16-Q5-E32", emb_dtype="bf16", E=32, Q=5, N=(150, 9)),      # E not a multiple of 64:
+    dict(name="umma16-Q16-E16", emb_dtype="bf16", E=16, Q=16, N=(77,)),       # 16-byte-column tiles
 ]
 
 
