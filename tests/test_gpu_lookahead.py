@@ -77,7 +77,9 @@ ATTN_CASES = [
     dict(B=2, N=(40, 72), k=(5, 9), C=64, Q=64, H=4),       # runs of 5 and 9 tiles
     dict(B=2, N=(40, 72), k=(5, 9), C=16, Q=64, H=4),       # 4 chunks a tile; ragged last tiles
     dict(B=2, N=(30, 50), k=(7, 3), C=32, Q=64, H=2),
-    dict(B=2, N=(12, 20), k=(3, 5), C=128, Q=64, H=2),      # 2 tiles a chunk
+    dict(B=2, N=(12, 20), k=(3, 5), C=128, Q=64, H=2),      # one tile a chunk
+    dict(B=2, N=(9, 6), k=(4, 1), C=256, Q=64, H=2),        # 2 tiles a chunk
+    dict(B=1, N=(5,), k=(3,), C=1024, Q=40, H=2),           # 8 tiles a chunk
     dict(B=2, N=(64, 40), k=(11, 1), C=8, Q=64, H=2),       # 8 chunks a tile; a 1-chunk sequence
     dict(B=2, N=(40, 72), k=(5, 9), C=64, Q=13, H=4),       # a partial window
     dict(B=1, N=(40,), k=(6,), C=64, Q=1, H=8),             # a single query
