@@ -14,7 +14,9 @@
 //
 // One CTA per SM, persistent over a balanced run of tiles:
 //  * A tile is 128 consecutive kept tokens of one (sequence, head). The tiles of all (b, h)
-//    form one global list; CTA c takes tiles [c*S/G, (c+1)*S/G) (split-K over the list).
+//    form one global list split over the CTAs by cost (split-K over the list): a tile costs 1
+//    and the start of a (b, h) run 4 more, since a CTA that switches runs reloads its queries
+//    and merges the finished run.
 //  * Warp 8 (producer) streams each tile's K and V rows from the full cache, through the
 //    kept chunk ids (or from a compact resident buffer), with 3-D TMA tile loads in the
 //    128-byte-swizzled layout the MMAs read: a 2-deep K ring (a K tile is free once its S
@@ -90,6 +92,8 @@ struct LaParams {
     int32_t boxh;     // token rows per TMA box: min(C, 128)
     int32_t nbox;     // boxes per tile: 128 / boxh
     int64_t S;        // tiles in the global list
+    int64_t F;        // total cost of the list: S + W * (runs - 1)
+    int32_t W;        // extra cost of a run start, in tiles (its Q reload and run-end merge)
     float qscale;     // log2(e) / sqrt(Dh)
     int32_t tile_off[kMaxB + 1];  // first tile of each sequence (its H runs follow in head order)
 };
@@ -124,8 +128,28 @@ __device__ __forceinline__ void la_next(LaCursor& u, const SeqTable& tab, const 
     if (u.b + 1 < tab.B) la_seq(u, u.b + 1, tab);
 }
 
-__host__ __device__ __forceinline__ int64_t la_cta_of_tile(int64_t s, int64_t S, int G) {
-    return ((s + 1) * G + S - 1) / S - 1;
+// The tile list is split by cost, not by count: a tile costs 1 and the start of a (sequence,
+// head) run W more, so a CTA that switches runs (a Q reload and a run-end merge) gets fewer
+// tiles. Tile s goes to CTA floor(cost(s) * G / F), cost(s) = s + W * run(s), which increases
+// with s, so each CTA gets a contiguous range; W = 0 (small lists) is the even split.
+__device__ __forceinline__ int64_t la_run_of(int64_t s, const SeqTable& tab, const LaParams& lp) {
+    const int b = seq_of(lp.tile_off, tab.B, s);
+    const int nt = ((tab.kept_off[b + 1] - tab.kept_off[b]) * tab.C + la::kTile - 1) / la::kTile;
+    return (int64_t)b * lp.H + (s - lp.tile_off[b]) / nt;
+}
+
+__device__ __forceinline__ int la_cta_of(int64_t s, const SeqTable& tab, const LaParams& lp) {
+    return (int)((s + (int64_t)lp.W * la_run_of(s, tab, lp)) * lp.G / lp.F);
+}
+
+// First tile of CTA c (c = G gives S): the least s with la_cta_of(s) >= c.
+__device__ __forceinline__ int64_t la_cta_start(int c, const SeqTable& tab, const LaParams& lp) {
+    int64_t lo = 0, hi = lp.S;
+    while (lo < hi) {
+        const int64_t mid = (lo + hi) >> 1;
+        if (la_cta_of(mid, tab, lp) >= c) hi = mid; else lo = mid + 1;
+    }
+    return lo;
 }
 
 // Token row (in the K/V tensor) of box j of global tile s. A box past the sequence's kept
@@ -304,11 +328,10 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     __shared__ int s_abort;
     __shared__ float2 s_ml1[kRows];  // group 1's (m, l) per row, at a run end
     __shared__ float2 s_mlh[kQmax];  // merged (m, l) of rows 64..127, at a run end
+    __shared__ int64_t s_range[2];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x;
-    const int64_t s0 = (int64_t)c * lp.S / lp.G, s1 = (int64_t)(c + 1) * lp.S / lp.G;
-    const int n = (int)(s1 - s0);  // tiles of this CTA (the list is below 2^31 tiles)
     const uint32_t raw = smem_u32(la_raw);
     const uint32_t sQ = (raw + 1023u) & ~1023u;
     const uint32_t sX = sQ + kQBytes, sK = sX + kScratch, sV = sK + kKStages * kOperand;
@@ -335,6 +358,8 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         mbar_init(endb, 1);
         fence_mbar_init();
         s_abort = 0;
+        s_range[0] = la_cta_start(c, tab, lp);
+        s_range[1] = la_cta_start(c + 1, tab, lp);
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
@@ -346,6 +371,8 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     __syncthreads();
     la_fence_after();
     const uint32_t tmem = s_tmem;
+    const int64_t s0 = s_range[0], s1 = s_range[1];
+    const int n = (int)(s1 - s0);  // tiles of this CTA (the list is below 2^31 tiles)
     pdl_trigger();
 
     if (warp == kProducerWarp) {
@@ -755,11 +782,11 @@ k_attn_la_merge(const float* __restrict__ part_o, const float* __restrict__ part
     const int kt = (tab.kept_off[b + 1] - tab.kept_off[b]) * tab.C;
     const int nt = (kt + la::kTile - 1) / la::kTile;
     const int64_t ts = lp.tile_off[b] + (int64_t)h * nt, te = ts + nt;
-    const int c0 = (int)la_cta_of_tile(ts, lp.S, lp.G), c1 = (int)la_cta_of_tile(te - 1, lp.S, lp.G);
+    const int c0 = la_cta_of(ts, tab, lp), c1 = la_cta_of(te - 1, tab, lp);
     if (c0 == c1) return;  // written directly by its CTA
     const int ns = c1 - c0 + 1;
     // the run is the first run of every CTA after c0; of c0 only if c0's tiles start inside it
-    const int slot0 = 2 * c0 + (((int64_t)c0 * lp.S / lp.G) >= ts ? 0 : 1);
+    const int slot0 = 2 * c0 + (la_cta_start(c0, tab, lp) >= ts ? 0 : 1);
     auto slot_of = [&](int i) { return i == 0 ? slot0 : 2 * (c0 + i); };
 
     float M = -INFINITY;
@@ -881,6 +908,10 @@ cudaError_t launch_attention_la(const lsa_dims& d, const SeqTable& tab, int max_
     lp.tile_off[d.B] = (int32_t)S;
     lp.S = S;
     lp.G = (int)(S < max_ctas ? S : max_ctas);
+    // a run switch costs about 4 tiles (measured); with at least 16 tiles per CTA no CTA can be
+    // left empty by the weighting, below that the split is even
+    lp.W = S >= 16 * (int64_t)lp.G ? 4 : 0;
+    lp.F = S + (int64_t)lp.W * ((int64_t)d.B * d.H - 1);
     lp.indexed = ids != nullptr ? 1 : 0;
     lp.qscale = 1.4426950408889634f / sqrtf((float)kDh);
 
