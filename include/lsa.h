@@ -204,6 +204,22 @@ LSA_API lsa_status lsa_decode_step_lookahead(const lsa_dims *dims, const void *q
                                              int32_t *chunk_ids_out, float *out, float *lse, void *ws,
                                              size_t ws_bytes, void *stream);
 
+/* The split of the lookahead attention's tile list over its CTAs, exactly as
+ * lsa_sparse_decode_attn_lookahead uses it. Host only: no device call, no GPU needed.
+ * The list holds, for each sequence b and then each head h, ceil(k_b * C / 128) tiles of
+ * 128 kept tokens (one (sequence, head) run). A tile costs 1 and the start of a run 4 more;
+ * CTA c takes the contiguous tiles whose cost lies in [ceil(c*F/G), ceil((c+1)*F/G)), with
+ * F the total cost and G = min(tiles, max_ctas, 256). Where that would leave a CTA without
+ * tiles, every tile costs 1 (the even split).
+ *   max_ctas   CTAs to split over (the attention launches one per SM), >= 1
+ *   cta_start  host array of at least min(max_ctas, 256) + 1 int32: the first tile of each
+ *              CTA, then cta_start[G] = the number of tiles
+ *   n_ctas     host int32, receives G
+ * Errors: LSA_ERR_INVALID_ARG (bad dims, null pointer, max_ctas < 1), LSA_ERR_UNSUPPORTED
+ * (a shape the lookahead attention does not take). */
+LSA_API lsa_status lsa_lookahead_partition(const lsa_dims *dims, int32_t max_ctas, int32_t *cta_start,
+                                           int32_t *n_ctas);
+
 /* Retrieval cycle of the lookahead loop [R3-2.3 steps 4-7; review section 3-1: the
  * indexer re-scores about every 64 decode steps and attention runs over the kept
  * chunks until the next cycle]. Scores every chunk, keeps the top-k, and refreshes a

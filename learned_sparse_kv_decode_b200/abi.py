@@ -62,6 +62,8 @@ def _load():
         "lsa_sparse_decode_attn_lookahead": ([dp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "lsa_decode_step_lookahead": ([dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "lsa_get_device_status": ([vp, vp], ctypes.c_int),
+        "lsa_lookahead_partition": ([dp, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)],
+                                    ctypes.c_int),
         "lsa_sparse_decode_attn_noalloc": ([dp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "lsa_refresh_resident": ([dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "lsa_threshold_select": ([dp, vp, ctypes.c_float, ctypes.c_int32, vp, vp, vp, sz, vp], ctypes.c_int),
@@ -197,6 +199,15 @@ def lsa_decode_step_lookahead(dims, q_emb, chunk_emb, q, K, V, chunk_ids_out, ou
     _check(lib.lsa_decode_step_lookahead(dims.ptr, _p(q_emb), _p(chunk_emb), _p(q), _p(K), _p(V),
                                          _p(chunk_ids_out), _p(out), _p(lse), _p(ws), _nbytes(ws),
                                          _stream(stream)), "lsa_decode_step_lookahead")
+
+
+def lsa_lookahead_partition(dims, max_ctas: int) -> list:
+    """First tile of each CTA of the lookahead attention's split, then the tile count (host only)."""
+    n = min(int(max_ctas), 256) + 1 if max_ctas >= 1 else 1
+    starts = (ctypes.c_int32 * n)()
+    g = ctypes.c_int32(0)
+    _check(lib.lsa_lookahead_partition(dims.ptr, int(max_ctas), starts, ctypes.byref(g)), "lsa_lookahead_partition")
+    return list(starts[:g.value + 1])
 
 
 def lsa_indexer_score_fp8(dims, n_layers, n_heads, ensemble, compressed_k, q_fp8, q_scale, head_w, scores, ws,

@@ -78,6 +78,8 @@ constexpr int kSBufs = 2;                 // S buffers in TMEM (one per softmax 
 constexpr uint32_t kTmemCols = 512;       // S: 2 x 128 columns, then O of group 0 and of group 1
 constexpr uint32_t kTmemO = kSBufs * kTile;  // first O column (group 0; group 1 follows)
 constexpr float kRescale = 8.0f;          // lazy-rescale threshold (log2 units)
+constexpr int kMaxCtas = 256;             // CTAs of one launch (one per SM)
+constexpr int kRunCost = 4;               // extra cost of a run start in the tile split, in tiles (measured)
 constexpr float kLn2 = 0.69314718055994531f;
 static_assert(kQBytes % 1024 == 0 && kScratch % 1024 == 0 && kOperand % 1024 == 0, "1 KiB swizzle atoms");
 static_assert(kTmemO + 2 * 128 == kTmemCols, "TMEM: S buffers then two O accumulators");
@@ -92,10 +94,9 @@ struct LaParams {
     int32_t boxh;     // token rows per TMA box: min(C, 128)
     int32_t nbox;     // boxes per tile: 128 / boxh
     int64_t S;        // tiles in the global list
-    int64_t F;        // total cost of the list: S + W * (runs - 1)
-    int32_t W;        // extra cost of a run start, in tiles (its Q reload and run-end merge)
     float qscale;     // log2(e) / sqrt(Dh)
-    int32_t tile_off[kMaxB + 1];  // first tile of each sequence (its H runs follow in head order)
+    int32_t tile_off[kMaxB + 1];        // first tile of each sequence (its H runs follow in head order)
+    int32_t cta_start[la::kMaxCtas + 1];  // first tile of each CTA; cta_start[G] = S
 };
 
 // Position in the tile list: run (b, h), tile t of the run.
@@ -128,26 +129,12 @@ __device__ __forceinline__ void la_next(LaCursor& u, const SeqTable& tab, const 
     if (u.b + 1 < tab.B) la_seq(u, u.b + 1, tab);
 }
 
-// The tile list is split by cost, not by count: a tile costs 1 and the start of a (sequence,
-// head) run W more, so a CTA that switches runs (a Q reload and a run-end merge) gets fewer
-// tiles. Tile s goes to CTA floor(cost(s) * G / F), cost(s) = s + W * run(s), which increases
-// with s, so each CTA gets a contiguous range; W = 0 (small lists) is the even split.
-__device__ __forceinline__ int64_t la_run_of(int64_t s, const SeqTable& tab, const LaParams& lp) {
-    const int b = seq_of(lp.tile_off, tab.B, s);
-    const int nt = ((tab.kept_off[b + 1] - tab.kept_off[b]) * tab.C + la::kTile - 1) / la::kTile;
-    return (int64_t)b * lp.H + (s - lp.tile_off[b]) / nt;
-}
-
-__device__ __forceinline__ int la_cta_of(int64_t s, const SeqTable& tab, const LaParams& lp) {
-    return (int)((s + (int64_t)lp.W * la_run_of(s, tab, lp)) * lp.G / lp.F);
-}
-
-// First tile of CTA c (c = G gives S): the least s with la_cta_of(s) >= c.
-__device__ __forceinline__ int64_t la_cta_start(int c, const SeqTable& tab, const LaParams& lp) {
-    int64_t lo = 0, hi = lp.S;
+// The CTA that owns tile s: the last c with cta_start[c] <= s (the ranges are non-empty).
+__device__ __forceinline__ int la_cta_of(int64_t s, const LaParams& lp) {
+    int lo = 0, hi = lp.G - 1;
     while (lo < hi) {
-        const int64_t mid = (lo + hi) >> 1;
-        if (la_cta_of(mid, tab, lp) >= c) hi = mid; else lo = mid + 1;
+        const int mid = (lo + hi + 1) >> 1;
+        if (lp.cta_start[mid] <= s) lo = mid; else hi = mid - 1;
     }
     return lo;
 }
@@ -328,7 +315,6 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     __shared__ int s_abort;
     __shared__ float2 s_ml1[kRows];  // group 1's (m, l) per row, at a run end
     __shared__ float2 s_mlh[kQmax];  // merged (m, l) of rows 64..127, at a run end
-    __shared__ int64_t s_range[2];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x;
@@ -358,8 +344,6 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         mbar_init(endb, 1);
         fence_mbar_init();
         s_abort = 0;
-        s_range[0] = la_cta_start(c, tab, lp);
-        s_range[1] = la_cta_start(c + 1, tab, lp);
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
@@ -371,7 +355,7 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     __syncthreads();
     la_fence_after();
     const uint32_t tmem = s_tmem;
-    const int64_t s0 = s_range[0], s1 = s_range[1];
+    const int64_t s0 = lp.cta_start[c], s1 = lp.cta_start[c + 1];
     const int n = (int)(s1 - s0);  // tiles of this CTA (the list is below 2^31 tiles)
     pdl_trigger();
 
@@ -782,11 +766,11 @@ k_attn_la_merge(const float* __restrict__ part_o, const float* __restrict__ part
     const int kt = (tab.kept_off[b + 1] - tab.kept_off[b]) * tab.C;
     const int nt = (kt + la::kTile - 1) / la::kTile;
     const int64_t ts = lp.tile_off[b] + (int64_t)h * nt, te = ts + nt;
-    const int c0 = la_cta_of(ts, tab, lp), c1 = la_cta_of(te - 1, tab, lp);
+    const int c0 = la_cta_of(ts, lp), c1 = la_cta_of(te - 1, lp);
     if (c0 == c1) return;  // written directly by its CTA
     const int ns = c1 - c0 + 1;
     // the run is the first run of every CTA after c0; of c0 only if c0's tiles start inside it
-    const int slot0 = 2 * c0 + (la_cta_start(c0, tab, lp) >= ts ? 0 : 1);
+    const int slot0 = 2 * c0 + (lp.cta_start[c0] == ts ? 0 : 1);
     auto slot_of = [&](int i) { return i == 0 ? slot0 : 2 * (c0 + i); };
 
     float M = -INFINITY;
@@ -878,18 +862,63 @@ cudaError_t la_init_attrs(int* ctas_per_sm) {
     return cudaSuccess;
 }
 
-// Tiles of the global list (sum over sequences of H * ceil(k_b * C / 64)).
+// Tiles of one (sequence, head) run of kt kept tokens.
+static int64_t la_run_tiles(int64_t kt) { return (kt + la::kTile - 1) / la::kTile; }
+
+// Tiles of the global list (sum over sequences of H * ceil(k_b * C / 128)).
 int64_t la_tiles(const lsa_dims& d, const SeqTable& tab) {
     int64_t S = 0;
-    for (int b = 0; b < d.B; ++b) {
-        const int64_t kt = (int64_t)(tab.kept_off[b + 1] - tab.kept_off[b]) * tab.C;
-        S += (int64_t)d.H * ((kt + la::kTile - 1) / la::kTile);
-    }
+    for (int b = 0; b < d.B; ++b)
+        S += (int64_t)d.H * la_run_tiles((int64_t)(tab.kept_off[b + 1] - tab.kept_off[b]) * tab.C);
     return S;
 }
 
 // q [B][Qw][H][Dh], K/V [kv_rows][H][Dh] bf16; ids (or nullptr: compact resident buffers);
 // part_o [2*max_ctas][Qw][Dh] and part_ml [2*max_ctas][Qw][2] fp32 workspace.
+// Split of the global tile list over the CTAs, by cost rather than by count: a tile costs 1
+// and the start of a (sequence, head) run W more (its query reload and run-end merge take about
+// as long as W tiles), so a CTA that opens a run takes fewer tiles. cost(s) = s + W * run(s)
+// increases with s; CTA c takes the tiles with ceil(c F / G) <= cost < ceil((c + 1) F / G),
+// F = S + W (runs - 1), one contiguous range each. A split that would leave a CTA empty (short
+// lists) falls back to the even split (W = 0). Writes cta_start[0..G] and returns G.
+int la_partition(const SeqTable& tab, int H, int max_ctas, int32_t* cta_start) {
+    int64_t S = 0;
+    for (int b = 0; b < tab.B; ++b)
+        S += (int64_t)H * la_run_tiles((int64_t)(tab.kept_off[b + 1] - tab.kept_off[b]) * tab.C);
+    int G = (int)(S < max_ctas ? S : max_ctas);
+    if (G > la::kMaxCtas) G = la::kMaxCtas;
+    const int64_t runs = (int64_t)tab.B * H;
+    for (int W = la::kRunCost; W >= 0; W -= la::kRunCost) {
+        const int64_t F = S + W * (runs - 1);
+        int b = 0;
+        int64_t off = 0;  // first tile of sequence b
+        for (int c = 0; c <= G; ++c) {
+            const int64_t T = (c * F + G - 1) / G;  // least cost of CTA c
+            int64_t s = S;
+            for (; b < tab.B; ++b) {
+                const int64_t nt = la_run_tiles((int64_t)(tab.kept_off[b + 1] - tab.kept_off[b]) * tab.C);
+                const int64_t base = off + W * (int64_t)b * H;  // cost of the sequence's first tile
+                const int64_t last = base + (H - 1) * (nt + W) + nt - 1;
+                if (T <= last) {
+                    if (T <= base) {
+                        s = off;
+                    } else {
+                        const int64_t h = (T - base) / (nt + W), t = T - base - h * (nt + W);
+                        s = t < nt ? off + h * nt + t : off + (h + 1) * nt;
+                    }
+                    break;
+                }
+                off += (int64_t)H * nt;
+            }
+            cta_start[c] = (int32_t)s;
+        }
+        bool ok = true;
+        for (int c = 0; c < G; ++c) ok = ok && cta_start[c] < cta_start[c + 1];
+        if (ok || W == 0) break;
+    }
+    return G;
+}
+
 cudaError_t launch_attention_la(const lsa_dims& d, const SeqTable& tab, int max_ctas, const void* q, const void* K,
                                 const void* V, int64_t kv_rows, const int32_t* ids, float* part_o, float* part_ml,
                                 float* out, float* lse, uint32_t* err, cudaStream_t stream, bool pdl) {
@@ -907,11 +936,7 @@ cudaError_t launch_attention_la(const lsa_dims& d, const SeqTable& tab, int max_
     }
     lp.tile_off[d.B] = (int32_t)S;
     lp.S = S;
-    lp.G = (int)(S < max_ctas ? S : max_ctas);
-    // a run switch costs about 4 tiles (measured); with at least 16 tiles per CTA no CTA can be
-    // left empty by the weighting, below that the split is even
-    lp.W = S >= 16 * (int64_t)lp.G ? 4 : 0;
-    lp.F = S + (int64_t)lp.W * ((int64_t)d.B * d.H - 1);
+    lp.G = la_partition(tab, d.H, max_ctas, lp.cta_start);
     lp.indexed = ids != nullptr ? 1 : 0;
     lp.qscale = 1.4426950408889634f / sqrtf((float)kDh);
 

@@ -51,6 +51,7 @@ cudaError_t launch_refresh(const lsa_dims& d, const SeqTable& tab, int max_n, co
 cudaError_t la_init_attrs(int* ctas_per_sm);
 int la_max_queries();
 int64_t la_tiles(const lsa_dims& d, const SeqTable& tab);
+int la_partition(const SeqTable& tab, int H, int max_ctas, int32_t* cta_start);
 cudaError_t launch_attention_la(const lsa_dims& d, const SeqTable& tab, int max_ctas, const void* q, const void* K,
                                 const void* V, int64_t kv_rows, const int32_t* ids, float* part_o, float* part_ml,
                                 float* out, float* lse, uint32_t* err, cudaStream_t stream, bool pdl);
@@ -361,6 +362,18 @@ lsa_status lsa_sparse_decode_attn_lookahead(const lsa_dims* dims, const void* q,
                                            reinterpret_cast<float*>(at(ws, w.la_ml)), out, lse,
                                            reinterpret_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream),
                                            true));
+}
+
+lsa_status lsa_lookahead_partition(const lsa_dims* dims, int32_t max_ctas, int32_t* cta_start, int32_t* n_ctas) {
+    if (cta_start == nullptr || n_ctas == nullptr || max_ctas < 1) return LSA_ERR_INVALID_ARG;
+    Prepared p;
+    lsa_status s = prepare(dims, &p);
+    if (s != LSA_OK) return s;
+    int64_t kv_rows = 0;
+    s = la_check(dims, p, false, &kv_rows);
+    if (s != LSA_OK) return s;
+    *n_ctas = la_partition(p.tab, dims->H, max_ctas, cta_start);
+    return LSA_OK;
 }
 
 lsa_status lsa_decode_step_lookahead(const lsa_dims* dims, const void* q_emb, const void* chunk_emb, const void* q,

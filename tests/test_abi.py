@@ -14,7 +14,7 @@ from learned_sparse_kv_decode_b200 import abi  # noqa: E402
 
 def test_exports_every_header_symbol():
     names = lsa.header_symbols()
-    assert len(names) == 22
+    assert len(names) == 23
     for n in names:
         assert hasattr(abi.lib, n), n
 
