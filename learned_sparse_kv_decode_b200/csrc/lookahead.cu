@@ -773,40 +773,39 @@ k_attn_la_merge(const float* __restrict__ part_o, const float* __restrict__ part
     const int slot0 = 2 * c0 + (lp.cta_start[c0] == ts ? 0 : 1);
     auto slot_of = [&](int i) { return i == 0 ? slot0 : 2 * (c0 + i); };
 
-    float M = -INFINITY;
-    for (int i = lane; i < ns; i += 32) M = fmaxf(M, part_ml[((int64_t)slot_of(i) * lp.Qw + q) * 2]);
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float L = 0.f;
+    // chunks of up to 16 pieces, each one round trip: lane i loads (m, l) of piece i of the chunk
+    // while every lane loads its 4 columns of all the chunk's rows; the running max rescales
+    float M = -INFINITY, L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    constexpr int kU = 8;  // partial rows in flight per lane
-    for (int i0 = 0; i0 < ns; i0 += 32) {
-        float wgt = 0.f;
-        if (i0 + lane < ns) {
-            const float2 ml = *reinterpret_cast<const float2*>(part_ml + ((int64_t)slot_of(i0 + lane) * lp.Qw + q) * 2);
-            wgt = ml.x == -INFINITY ? 0.f : la_ex2(ml.x - M);
-            L = fmaf(wgt, ml.y, L);
-        }
-        const int cnt = ns - i0 < 32 ? ns - i0 : 32;
-        for (int j0 = 0; j0 < cnt; j0 += kU) {
-            float4 v[kU];
+    constexpr int kU = 16;  // partial rows in flight per lane
+    for (int i0 = 0; i0 < ns; i0 += kU) {
+        const int cnt = ns - i0 < kU ? ns - i0 : kU;
+        float2 ml = make_float2(-INFINITY, 0.f);
+        if (lane < cnt) ml = *reinterpret_cast<const float2*>(part_ml + ((int64_t)slot_of(i0 + lane) * lp.Qw + q) * 2);
+        float4 v[kU];  // rows past the chunk reload its last row (weight 0), so every load is issued
 #pragma unroll
-            for (int u = 0; u < kU; ++u)
-                v[u] = j0 + u < cnt ? *reinterpret_cast<const float4*>(
-                                          part_o + ((int64_t)slot_of(i0 + j0 + u) * lp.Qw + q) * kDh + lane * 4)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < kU; ++u)
+            v[u] = *reinterpret_cast<const float4*>(
+                part_o + ((int64_t)slot_of(i0 + (u < cnt ? u : cnt - 1)) * lp.Qw + q) * kDh + lane * 4);
+        float mc = ml.x;
+        for (int off = 16; off > 0; off >>= 1) mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, off));
+        const float Mn = fmaxf(M, mc);
+        const float a = M == -INFINITY ? 0.f : la_ex2(M - Mn);  // rescale of the earlier chunks
+        const float wgt = ml.x == -INFINITY ? 0.f : la_ex2(ml.x - Mn);
+        float lc = wgt * ml.y;
+        for (int off = 16; off > 0; off >>= 1) lc += __shfl_xor_sync(0xffffffffu, lc, off);
+        L = fmaf(L, a, lc);
+        acc = make_float4(acc.x * a, acc.y * a, acc.z * a, acc.w * a);
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const float wj = __shfl_sync(0xffffffffu, wgt, (j0 + u) & 31);
-                if (j0 + u < cnt) {
-                    acc.x = fmaf(wj, v[u].x, acc.x);
-                    acc.y = fmaf(wj, v[u].y, acc.y);
-                    acc.z = fmaf(wj, v[u].z, acc.z);
-                    acc.w = fmaf(wj, v[u].w, acc.w);
-                }
-            }
+        for (int u = 0; u < kU; ++u) {
+            const float wj = u < cnt ? __shfl_sync(0xffffffffu, wgt, u) : 0.f;
+            acc.x = fmaf(wj, v[u].x, acc.x);
+            acc.y = fmaf(wj, v[u].y, acc.y);
+            acc.z = fmaf(wj, v[u].z, acc.z);
+            acc.w = fmaf(wj, v[u].w, acc.w);
         }
+        M = Mn;
     }
-    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
     const float inv = 1.f / L;
     float* dst = out + (((int64_t)b * lp.Qw + q) * lp.H + h) * kDh + lane * 4;
     *reinterpret_cast<float4*>(dst) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
