@@ -12,11 +12,12 @@
 // element, 64 flop per byte at Qw = 64. That is still HBM-bound on the tensor pipe, but far
 // beyond what the CUDA cores sustain at HBM speed, so both products run as tcgen05 MMAs.
 //
-// One CTA per SM, persistent over a balanced run of tiles:
+// One CTA per SM, persistent over one contiguous range of tiles:
 //  * A tile is 128 consecutive kept tokens of one (sequence, head). The tiles of all (b, h)
 //    form one global list split over the CTAs by cost (split-K over the list): a tile costs 1
 //    and the start of a (b, h) run 4 more, since a CTA that switches runs reloads its queries
-//    and merges the finished run.
+//    and merges the finished run. The host computes the ranges (la_partition) and passes them
+//    in the kernel parameters.
 //  * Warp 8 (producer) streams each tile's K and V rows from the full cache, through the
 //    kept chunk ids (or from a compact resident buffer), with 3-D TMA tile loads in the
 //    128-byte-swizzled layout the MMAs read: a 2-deep K ring (a K tile is free once its S
