@@ -327,88 +327,85 @@ k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
 
 // Merge of the split partials of one (sequence, head) with the log-sum-exp rule.
 // grid (B, H, kMergeDimSplit): a CTA merges kMergeDims of the Dh output columns over all of the
-// sequence's slots; kMergeGroups thread groups share the slots so that many loads are in flight.
+// sequence's slots. Warp g takes slots g, g + 8, ...; lane k owns column k of the CTA's 32. Each
+// pass issues kMergeU slots' (m, l) and partial column together (one round trip) and folds them
+// into the warp's running (m, l, acc); the eight warps are then combined in shared memory.
 constexpr int kMergeDimSplit = 4;
 constexpr int kMergeDims = kDh / kMergeDimSplit;          // 32 columns per CTA
 constexpr int kMergeThreads = 256;
-constexpr int kMergeGroups = kMergeThreads / kMergeDims;  // 8 slot groups
-constexpr int kMergeUnroll = 8;
-constexpr int kMergeMaxSlots = 2048;
+constexpr int kMergeGroups = kMergeThreads / kMergeDims;  // 8 slot groups (one warp each)
+constexpr int kMergeU = 16;                               // slots in flight per thread
+static_assert(kMergeDims == 32, "one lane per column");
 
 __global__ void __launch_bounds__(kMergeThreads)
 k_attn_merge(const float* __restrict__ part_o, const float* __restrict__ part_ml,
              float* __restrict__ out, float* __restrict__ lse, const SeqTable tab,
              const AttnParams ap) {
-    __shared__ float s_w[kMergeMaxSlots];
-    __shared__ float s_red[kMergeThreads / 32];
+    __shared__ float s_m[kMergeGroups], s_l[kMergeGroups];
     __shared__ float s_acc[kMergeGroups][kMergeDims];
-    const int b = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, g = tid >> 5;
     pdl_wait();
     const int64_t st0 = (int64_t)tab.kept_off[b] * ap.SPC;
     const int64_t st1 = (int64_t)tab.kept_off[b + 1] * ap.SPC - 1;
     const int c_lo = (int)cta_of_stage(st0, ap.S, ap.G);
-    const int ns = (int)cta_of_stage(st1, ap.S, ap.G) - c_lo + 1;
+    const int ns = (int)cta_of_stage(st1, ap.S, ap.G) - c_lo + 1;  // >= 1
     const uint64_t slot0 = (uint64_t)c_lo + b;
+    const int d = blockIdx.z * kMergeDims + lane;
+    const uint64_t sstride = (uint64_t)ap.H * kDh;
+    const float* po = part_o + (slot0 * ap.H + h) * kDh + d;
+    const float* pm = part_ml + (slot0 * ap.H + h) * 2;
 
-    // 1. the running maxima m and sums l of all slots -> M
-    float mloc = -INFINITY;
-    for (int i = tid; i < ns; i += kMergeThreads) {
-        const float m = part_ml[((slot0 + i) * ap.H + h) * 2];
-        s_w[i] = m;
-        mloc = fmaxf(mloc, m);
-    }
-    for (int off = 16; off > 0; off >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, off));
-    if (lane == 0) s_red[warp] = mloc;
-    __syncthreads();
-    float M = s_red[0];
+    float m = -INFINITY, l = 0.f, a = 0.f;  // this warp's slots so far (m, l uniform in the warp)
+    for (int i0 = g; i0 < ns; i0 += kMergeGroups * kMergeU) {
+        float v[kMergeU], mu[kMergeU], lu[kMergeU];
 #pragma unroll
-    for (int w = 1; w < kMergeThreads / 32; ++w) M = fmaxf(M, s_red[w]);
+        for (int u = 0; u < kMergeU; ++u) {  // past the last slot: reload it with no weight
+            const int i = i0 + u * kMergeGroups;
+            const int ic = i < ns ? i : ns - 1;
+            v[u] = po[(uint64_t)ic * sstride];
+            const float2 ml = *reinterpret_cast<const float2*>(pm + (uint64_t)ic * ap.H * 2);
+            mu[u] = i < ns ? ml.x : -INFINITY;
+            lu[u] = ml.y;
+        }
+        float mc = m;
+#pragma unroll
+        for (int u = 0; u < kMergeU; ++u) mc = fmaxf(mc, mu[u]);
+        if (mc == -INFINITY) continue;  // no weight yet (slots of a count of 0)
+        const float sc = m == -INFINITY ? 0.f : ex2(m - mc);
+        l *= sc;
+        a *= sc;
+#pragma unroll
+        for (int u = 0; u < kMergeU; ++u) {
+            const float w = mu[u] == -INFINITY ? 0.f : ex2(mu[u] - mc);
+            l = fmaf(w, lu[u], l);
+            a = fmaf(w, v[u], a);
+        }
+        m = mc;
+    }
+    if (lane == 0) {
+        s_m[g] = m;
+        s_l[g] = l;
+    }
+    s_acc[g][lane] = a;
+    __syncthreads();
+    if (g != 0) return;
+    float M = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kMergeGroups; ++k) M = fmaxf(M, s_m[k]);
     if (M == -INFINITY) {  // no kept token at all (a count of 0): empty output, lse = -inf
-        if (threadIdx.x < kMergeDims) out[((uint64_t)b * ap.H + h) * kDh + blockIdx.z * kMergeDims + threadIdx.x] = 0.f;
-        if (lse != nullptr && threadIdx.x == 0 && blockIdx.z == 0) lse[(uint64_t)b * ap.H + h] = -INFINITY;
+        out[((uint64_t)b * ap.H + h) * kDh + d] = 0.f;
+        if (lse != nullptr && d == 0) lse[(uint64_t)b * ap.H + h] = -INFINITY;
         return;
     }
-    // 2. slot weights 2^(m_s - M) and the merged denominator L
-    float lloc = 0.f;
-    for (int i = tid; i < ns; i += kMergeThreads) {
-        const float w = ex2(s_w[i] - M);
-        s_w[i] = w;
-        lloc = fmaf(part_ml[((slot0 + i) * ap.H + h) * 2 + 1], w, lloc);
+    float A = 0.f, L = 0.f;
+#pragma unroll
+    for (int k = 0; k < kMergeGroups; ++k) {
+        const float w = s_m[k] == -INFINITY ? 0.f : ex2(s_m[k] - M);
+        A = fmaf(w, s_acc[k][lane], A);
+        L = fmaf(w, s_l[k], L);
     }
-    for (int off = 16; off > 0; off >>= 1) lloc += __shfl_xor_sync(0xffffffffu, lloc, off);
-    __syncthreads();  // every thread has read s_red (M) before it is reused
-    if (lane == 0) s_red[warp] = lloc;
-    __syncthreads();
-    float L = 0.f;
-#pragma unroll
-    for (int w = 0; w < kMergeThreads / 32; ++w) L += s_red[w];
-    // 3. weighted sum of the partial outputs: group g takes slots g, g + groups, ...
-    const int g = tid / kMergeDims, dl = tid % kMergeDims, d = blockIdx.z * kMergeDims + dl;
-    const float* po = part_o + (slot0 * ap.H + h) * kDh + d;
-    const uint64_t sstride = (uint64_t)ap.H * kDh;
-    float a = 0.f;
-    for (int i0 = g; i0 < ns; i0 += kMergeGroups * kMergeUnroll) {
-        float v[kMergeUnroll];
-#pragma unroll
-        for (int u = 0; u < kMergeUnroll; ++u) {
-            const int i = i0 + u * kMergeGroups;
-            v[u] = i < ns ? po[(uint64_t)i * sstride] : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < kMergeUnroll; ++u) {
-            const int i = i0 + u * kMergeGroups;
-            if (i < ns) a = fmaf(v[u], s_w[i], a);
-        }
-    }
-    s_acc[g][dl] = a;
-    __syncthreads();
-    if (g == 0) {
-        float A = 0.f;
-#pragma unroll
-        for (int k = 0; k < kMergeGroups; ++k) A += s_acc[k][dl];
-        out[((uint64_t)b * ap.H + h) * kDh + d] = A / L;
-        if (lse != nullptr && d == 0) lse[(uint64_t)b * ap.H + h] = (M + log2f(L)) * 0.69314718055994531f;
-    }
+    out[((uint64_t)b * ap.H + h) * kDh + d] = A / L;
+    if (lse != nullptr && d == 0) lse[(uint64_t)b * ap.H + h] = (M + log2f(L)) * 0.69314718055994531f;
 }
 
 // ------------------------------------------------------------------ host side
@@ -517,7 +514,6 @@ cudaError_t launch_attention(const lsa_dims& d, const SeqTable& tab, int ctas_pe
     cfg.blockDim = dim3(kAttnThreads, 1, 1);
     cfg.dynamicSmemBytes = L.smem;
     if (L.tpg != 1 && L.tpg != 2 && L.tpg != 4 && L.tpg != 8) return cudaErrorInvalidValue;
-    if ((int64_t)L.ap.G > kMergeMaxSlots) return cudaErrorInvalidValue;
     cudaError_t e = d.kv_dtype == LSA_BF16
                         ? launch_split<true>(&cfg, L.tpg, q, K, V, ids, part_o, part_ml, tab, L.ap, err, counts)
                         : launch_split<false>(&cfg, L.tpg, q, K, V, ids, part_o, part_ml, tab, L.ap, err, counts);
