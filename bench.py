@@ -122,13 +122,19 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------- oracle sample
-def oracle_sample(w, seconds: float = None, steps: int = None, warmup: int = 0):
+REFERENCE_CAP_S = 150.0  # wall-clock bound of the reference arm's timed rounds
+
+
+def oracle_sample(w, seconds: float = None, steps: int = None, warmup: int = 0, cap: float = None):
     """Time the float64 oracle on a bounded sample of the workload and extrapolate to a step.
 
-    Work items, round robin: (a) chunk scores + top-k of one sequence, (b) exact attention of
-    one head over that sequence's kept tokens. A full step costs
-      sum_b [ t_score_per_chunk * N_b ] + sum_b [ t_attn_per_token * k_b * C * H ],
-    with both unit costs measured here. K/V rows are regenerated once, outside the timing."""
+    One round of the sample is, for each sampled sequence, (a) chunk scores + top-k of the
+    sequence and (b) exact attention of one head over its kept tokens, so every round measures
+    both unit costs. A full step costs
+      sum_b [ t_score_per_chunk * N_b ] + sum_b [ t_attn_per_token * k_b * C * H ].
+    `warmup` rounds are untimed. Then either `steps` rounds, stopping early once `cap` seconds
+    have passed (after at least one round), or rounds until `seconds` have passed. K/V rows are
+    regenerated once, outside the timing."""
     import numpy as np
 
     import datagen
@@ -148,41 +154,45 @@ def oracle_sample(w, seconds: float = None, steps: int = None, warmup: int = 0):
         Vh = datagen.kv_rows(w, "V", tok, [h]).astype(np.float64)
         qh = datagen.as_f32(x["q"][b], w.kv_dtype)[h:h + 1].astype(np.float64)
         prep.append((b, qf, ef, qh, Kh, Vh))
-    items = []
-    for p in prep:
-        items.append(("score", p))
-        items.append(("head", p))
     t_score, n_score, t_attn, n_attn = 0.0, 0, 0.0, 0
     scale = 1.0 / math.sqrt(w.Dh)
-    i = 0
+    rounds = 0
     t_begin = time.perf_counter()
+    t_timed = None
     while True:
-        kind, (b, qf, ef, qh, Kh, Vh) = items[i % len(items)]
-        t0 = time.perf_counter()
-        if kind == "score":
+        timed = rounds >= warmup
+        if timed and t_timed is None:
+            t_timed = time.perf_counter()
+        for b, qf, ef, qh, Kh, Vh in prep:
+            t0 = time.perf_counter()
             oracle.topk(oracle.chunk_scores(qf, ef), w.k[b])
-        else:
+            t1 = time.perf_counter()
             oracle.attention(qh, Kh, Vh, scale)
-        dt = time.perf_counter() - t0
-        if i >= warmup:
-            if kind == "score":
-                t_score += dt / w.N[b]
+            t2 = time.perf_counter()
+            if timed:
+                t_score += (t1 - t0) / w.N[b]
                 n_score += 1
-            else:
-                t_attn += dt / (w.k[b] * w.C)
+                t_attn += (t2 - t1) / (w.k[b] * w.C)
                 n_attn += 1
-        i += 1
-        if steps is not None and i >= steps + warmup:
+        rounds += 1
+        if not timed:
+            continue
+        done = rounds - warmup
+        now = time.perf_counter()
+        if steps is not None and (done >= steps or (cap is not None and now - t_timed >= cap)):
             break
-        if seconds is not None and time.perf_counter() - t_begin >= seconds and n_score and n_attn:
+        if steps is None and seconds is not None and now - t_begin >= seconds:
             break
-    per_chunk = t_score / max(n_score, 1)
-    per_token_head = t_attn / max(n_attn, 1)
+        if steps is None and seconds is None:
+            break
+    per_chunk = t_score / n_score
+    per_token_head = t_attn / n_attn
     t_step = sum(per_chunk * w.N[b] + per_token_head * w.k[b] * w.C * w.H for b in range(w.B))
-    sample = (f"{n_score} chunk-score+top-k items and {n_attn} one-head attention items on sequences "
-              f"{seqs}, float64 C oracle, 1 thread; step time extrapolated linearly to all {w.B} "
-              f"sequences x {w.H} heads")
-    return {"t_step": t_step, "items": i - warmup, "sample": sample, "elapsed": time.perf_counter() - t_begin}
+    sample = (f"{rounds - warmup} timed rounds (after {warmup} untimed), each one chunk-score+top-k item and "
+              f"one one-head attention item per sequence of {seqs}: {n_score} + {n_attn} items, float64 C "
+              f"oracle, 1 thread; step time extrapolated linearly to all {w.B} sequences x {w.H} heads")
+    return {"t_step": t_step, "rounds": rounds - warmup, "n_score": n_score, "n_attn": n_attn,
+            "sample": sample, "elapsed": time.perf_counter() - t_begin}
 
 
 def _oracle_sample_worker(args):
@@ -214,7 +224,7 @@ def run_reference(args):
         return 0
     import datagen
     w = datagen.workload(args.workload)
-    r = oracle_sample(w, steps=args.steps, warmup=args.warmup)
+    r = oracle_sample(w, steps=args.steps, warmup=args.warmup, cap=REFERENCE_CAP_S)
     value = 1.0 / r["t_step"]
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": args.gpus,

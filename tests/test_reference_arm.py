@@ -1,0 +1,47 @@
+"""CPU checks of bench.py's oracle sample (the reference arm and the cpu_baseline leg): every
+timed round measures both unit costs, so a short run cannot extrapolate a step from one kind
+of work alone, and the reference arm prints the contract's JSON line."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+import datagen  # noqa: E402
+
+
+@pytest.mark.parametrize("steps,warmup", [(1, 0), (1, 3), (2, 1)])
+def test_short_samples_time_both_kinds(steps, warmup):
+    w = datagen.workload("tiny")
+    r = bench.oracle_sample(w, steps=steps, warmup=warmup)
+    seqs = len({0, w.B - 1})
+    assert r["rounds"] == steps
+    assert r["n_score"] == steps * seqs and r["n_attn"] == steps * seqs
+    assert r["t_step"] > 0
+
+
+def test_time_bounded_sample():
+    w = datagen.workload("tiny")
+    r = bench.oracle_sample(w, seconds=0.2, warmup=1)
+    assert r["rounds"] >= 1 and r["n_score"] >= 1 and r["n_attn"] >= 1
+
+
+def test_cap_ends_a_long_request():
+    w = datagen.workload("tiny")
+    r = bench.oracle_sample(w, steps=10 ** 9, warmup=0, cap=0.3)
+    assert 1 <= r["rounds"] < 10 ** 9 and r["elapsed"] < 30
+
+
+def test_reference_arm_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                          "--steps", "2", "--warmup", "1"], capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "steps/s" and line["value"] > 0
+    assert line["steps"] == 2 and line["warmup"] == 1
+    assert line["e2e"]["value"] == line["value"] and line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and "2 timed rounds" in line["cpu_baseline"]["sample"]
