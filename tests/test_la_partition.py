@@ -95,3 +95,61 @@ def test_rejects(kw, status):
     with pytest.raises(lsa.LsaError) as e:
         lsa.lsa_lookahead_partition(d, kw.get("max_ctas", 148))
     assert e.value.status == status
+
+
+def _slots_written(starts, run_tiles):
+    """Slots the lookahead CTAs write for split runs: CTA c walks its tiles in order; a run it does
+    not hold whole goes to slot 2c if it is the CTA's first run, else 2c + 1."""
+    run_start = np.concatenate([[0], np.cumsum(run_tiles)])
+    written = {}
+    for c in range(len(starts) - 1):
+        s0, s1 = starts[c], starts[c + 1]
+        r = int(np.searchsorted(run_start, s0, side="right") - 1)
+        first = True
+        while r < len(run_tiles) and run_start[r] < s1:
+            whole = run_start[r] >= s0 and run_start[r + 1] <= s1
+            if not whole:
+                slot = 2 * c + (0 if first else 1)
+                assert slot not in written, "two pieces share a slot"
+                written[slot] = r
+            first = False
+            r += 1
+    return written, run_start
+
+
+def _slots_read(starts, run_start, r):
+    """Slots the merge kernel reads for run r: CTAs c0..c1 hold its pieces; piece 0 is c0's first
+    run only if c0 starts exactly at the run, and every later piece is that CTA's first run."""
+    cta_of = lambda s: int(np.searchsorted(starts[:-1], s, side="right") - 1)  # noqa: E731
+    ts, te = run_start[r], run_start[r + 1]
+    c0, c1 = cta_of(ts), cta_of(te - 1)
+    if c0 == c1:
+        return []
+    return [2 * c0 + (0 if starts[c0] == ts else 1)] + [2 * (c0 + i) for i in range(1, c1 - c0 + 1)]
+
+
+def _check_slots(starts, k, C, H):
+    run_tiles = [-(-kb * C // TILE) for kb in k for _ in range(H)]
+    written, run_start = _slots_written(starts, run_tiles)
+    read = {}
+    for r in range(len(run_tiles)):
+        for slot in _slots_read(starts, run_start, r):
+            assert slot not in read
+            read[slot] = r
+    assert read == written
+    assert all(slot < 2 * (len(starts) - 1) for slot in written)  # the workspace holds 2 slots per CTA
+
+
+@pytest.mark.parametrize("k,C,H,G", CASES, ids=[f"case{i}" for i in range(len(CASES))])
+def test_partial_slots_written_are_the_slots_merged(k, C, H, G):
+    _check_slots(lsa.lsa_lookahead_partition(_dims(k, C, H), G), k, C, H)
+
+
+def test_partial_slots_random_shapes():
+    rng = np.random.default_rng(9)
+    for _ in range(60):
+        B = int(rng.integers(1, 10))
+        C = int(2 ** rng.integers(3, 11))
+        H = int(2 ** rng.integers(0, 5))
+        k = [int(x) for x in rng.integers(1, 200, B)]
+        _check_slots(lsa.lsa_lookahead_partition(_dims(k, C, H), int(rng.integers(1, 200))), k, C, H)
