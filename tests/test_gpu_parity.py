@@ -4,7 +4,6 @@ Small cases are compared element by element (several tiles and ragged tails);
 the full-size decode workloads are run in the same launch configuration the
 benchmark times and compared on all chunk ids and on sampled (sequence, head)
 outputs, which the oracle recomputes from regenerated K/V rows."""
-import math
 
 import numpy as np
 import pytest
