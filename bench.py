@@ -195,6 +195,36 @@ def oracle_sample(w, seconds: float = None, steps: int = None, warmup: int = 0, 
             "sample": sample, "elapsed": time.perf_counter() - t_begin}
 
 
+DENSE_CONTEXT_MAX_TOKENS = 131072  # longest sequence timed in full by the dense context figure
+
+
+def oracle_dense_context(w) -> dict:
+    """Dense attention for context: the step the selection replaces, every head of every sequence
+    attending over all L_b tokens. The float64 oracle's attention of one head is timed (1 thread,
+    best of 3) over min(L_0, 131072) tokens and extrapolated linearly in tokens to all B sequences
+    x H heads. Its cost does not depend on the values, so K/V are drawn with numpy's generator
+    rather than regenerated from the workload's counter-based one (25 s at 128K on one core)."""
+    import numpy as np
+
+    import oracle
+
+    n = min(int(w.L[0]), DENSE_CONTEXT_MAX_TOKENS)
+    rng = np.random.default_rng(w.seed)
+    K = rng.standard_normal((n, 1, w.Dh))
+    V = rng.standard_normal((n, 1, w.Dh))
+    q = rng.standard_normal((1, w.Dh))
+    scale = 1.0 / math.sqrt(w.Dh)
+    best = float("inf")
+    for _ in range(3):
+        t0 = time.perf_counter()
+        oracle.attention(q, K, V, scale)
+        best = min(best, time.perf_counter() - t0)
+    t_step = best / n * sum(int(L) for L in w.L) * w.H
+    return {"value": 1.0 / t_step, "unit": "steps/s", "cores": 1, "kind": "oracle, dense attention (no selection)",
+            "sample": f"one head over {n} tokens, best of 3, float64 C oracle, 1 thread; extrapolated linearly "
+                      f"to {w.B} sequences x {w.H} heads over all {sum(int(L) for L in w.L)} tokens"}
+
+
 def _oracle_sample_worker(args):
     name, seconds = args
     import datagen
@@ -461,6 +491,7 @@ def run_ours(args):
         r = oracle_sample(w, seconds=args.cpu_seconds, warmup=2)
         cpu = {"value": 1.0 / r["t_step"], "unit": "steps/s", "cores": 1, "kind": "oracle", "sample": r["sample"]}
         cpu_all = oracle_sample_all_cores(w, args.cpu_seconds)
+        cpu_dense = oracle_dense_context(w)
     if rank == 0:
         e2e = hr["e2e"]
         line = {
@@ -509,6 +540,7 @@ def run_ours(args):
         if cpu is not None:
             line["cpu_baseline"] = cpu
             line["cpu_baseline_all_cores"] = cpu_all
+            line["cpu_dense_context"] = cpu_dense
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

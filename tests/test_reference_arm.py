@@ -45,3 +45,12 @@ def test_reference_arm_line():
     assert line["steps"] == 2 and line["warmup"] == 1
     assert line["e2e"]["value"] == line["value"] and line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["cpu_baseline"]["kind"] == "oracle" and "2 timed rounds" in line["cpu_baseline"]["sample"]
+
+
+def test_dense_context_costs_more_than_the_sparse_step():
+    # 128K keeps 12.5% of the tokens: the dense oracle step must be several times slower
+    w = datagen.workload("128k")
+    dense = bench.oracle_dense_context(w)
+    sparse = bench.oracle_sample(w, seconds=1.0, warmup=1)
+    assert dense["unit"] == "steps/s" and dense["cores"] == 1
+    assert dense["value"] * 3 < 1.0 / sparse["t_step"]
