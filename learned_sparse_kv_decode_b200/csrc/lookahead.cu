@@ -873,8 +873,6 @@ int64_t la_tiles(const lsa_dims& d, const SeqTable& tab) {
     return S;
 }
 
-// q [B][Qw][H][Dh], K/V [kv_rows][H][Dh] bf16; ids (or nullptr: compact resident buffers);
-// part_o [2*max_ctas][Qw][Dh] and part_ml [2*max_ctas][Qw][2] fp32 workspace.
 // Split of the global tile list over the CTAs, by cost rather than by count: a tile costs 1
 // and the start of a (sequence, head) run W more (its query reload and run-end merge take about
 // as long as W tiles), so a CTA that opens a run takes fewer tiles. cost(s) = s + W * run(s)
@@ -919,6 +917,8 @@ int la_partition(const SeqTable& tab, int H, int max_ctas, int32_t* cta_start) {
     return G;
 }
 
+// q [B][Qw][H][Dh], K/V [kv_rows][H][Dh] bf16; ids (or nullptr: compact resident buffers);
+// part_o [2*max_ctas][Qw][Dh] and part_ml [2*max_ctas][Qw][2] fp32 workspace.
 cudaError_t launch_attention_la(const lsa_dims& d, const SeqTable& tab, int max_ctas, const void* q, const void* K,
                                 const void* V, int64_t kv_rows, const int32_t* ids, float* part_o, float* part_ml,
                                 float* out, float* lse, uint32_t* err, cudaStream_t stream, bool pdl) {
