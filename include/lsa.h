@@ -205,7 +205,9 @@ LSA_API lsa_status lsa_decode_step_lookahead(const lsa_dims *dims, const void *q
                                              size_t ws_bytes, void *stream);
 
 /* The split of the lookahead attention's tile list over its CTAs, exactly as
- * lsa_sparse_decode_attn_lookahead uses it. Host only: no device call, no GPU needed.
+ * lsa_sparse_decode_attn_lookahead uses it. Host only: no device call, no GPU needed. This is
+ * not an operation of the method (the pages define none like it): it exposes how this library
+ * schedules the window attention [R3-2.3 steps 6-7], for tests and for callers sizing work.
  * The list holds, for each sequence b and then each head h, ceil(k_b * C / 128) tiles of
  * 128 kept tokens (one (sequence, head) run). A tile costs 1 and the start of a run 4 more;
  * CTA c takes the contiguous tiles whose cost lies in [ceil(c*F/G), ceil((c+1)*F/G)), with
