@@ -54,3 +54,33 @@ def test_dense_context_costs_more_than_the_sparse_step():
     sparse = bench.oracle_sample(w, seconds=1.0, warmup=1)
     assert dense["unit"] == "steps/s" and dense["cores"] == 1
     assert dense["value"] * 3 < 1.0 / sparse["t_step"]
+
+
+def _ranks_worker(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench._barrier(world)
+        q.put((rank, bench._max_over_ranks(1.5 + rank * 2.0, world)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo():
+    # the bench's timing is the maximum over ranks: every rank must report the slowest rank's time
+    import multiprocessing as mp
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_ranks_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert got == {0: 3.5, 1: 3.5}
