@@ -13,11 +13,13 @@ LIB = os.path.join(HERE, "libdatagen.so")
 def build(force: bool = False) -> str:
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
         return LIB
+    # one temporary per process: ranks that build at the same time do not share a file
+    tmp = f"{LIB}.{os.getpid()}.tmp"
     cmd = [os.environ.get("NVCC", "nvcc"), "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
            "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
-           SRC, "-o", LIB + ".tmp"]
+           SRC, "-o", tmp]
     subprocess.check_call(cmd)
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(tmp, LIB)  # atomic: a loader never sees a partial file
     return LIB
 
 

@@ -33,12 +33,14 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
         if os.path.getmtime(LIB) >= newest:
             return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
+    # one temporary per process: ranks that build at the same time do not share a file
+    tmp = f"{LIB}.{os.getpid()}.tmp"
     cmd = [nvcc, "-shared", *NVCC_FLAGS, *(extra_flags or []), "-I", INCLUDE, *_sources(),
-           "-o", LIB + ".tmp"]
+           "-o", tmp]
     if verbose:
         print(" ".join(cmd))
     subprocess.check_call(cmd)
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(tmp, LIB)  # atomic: a loader never sees a partial file
     return LIB
 
 

@@ -13,11 +13,13 @@ LIB = os.path.join(HERE, "liblsa_oracle.so")
 def build(force: bool = False) -> str:
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
         return LIB
+    # one temporary per process: ranks that build at the same time do not share a file
+    tmp = f"{LIB}.{os.getpid()}.tmp"
     # -ffp-contract=off: every multiply and add rounds on its own, as written.
     cmd = ["gcc", "-O2", "-std=c99", "-ffp-contract=off", "-fno-fast-math", "-shared", "-fPIC",
-           SRC, "-o", LIB + ".tmp", "-lm"]
+           SRC, "-o", tmp, "-lm"]
     subprocess.check_call(cmd)
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(tmp, LIB)  # atomic: a loader never sees a partial file
     return LIB
 
 
