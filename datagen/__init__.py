@@ -36,6 +36,7 @@ synthetic inputs stand in for them (no item of those suites is used).
 from __future__ import annotations
 
 import math
+import subprocess
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -304,14 +305,46 @@ def planted_positions(w: Workload, b: int) -> np.ndarray:
     return np.sort(perm[: w.plant_count[b]])
 
 
+_NATIVE_MIN = 1 << 16  # elements from which kv_rows uses the C generator
+_host = None
+
+
+def _host_lib():
+    """The C side of the generator (datagen/csrc/normal_host.c), built on first use; None
+    when it cannot be built (kv_rows then stays in numpy)."""
+    global _host
+    if _host is None:
+        import ctypes
+        try:
+            from . import build as _build
+            lib = ctypes.CDLL(_build.build_host())
+        except (OSError, subprocess.CalledProcessError):
+            _host = False
+            return None
+        i64, u32, vp = ctypes.c_int64, ctypes.c_uint32, ctypes.c_void_p
+        lib.dg_cache_rows.argtypes = [u32, u32, i64, i64, vp, i64, vp, i64, ctypes.c_int, vp]
+        lib.dg_cache_rows.restype = None
+        lib.dg_normal_f32.argtypes = [u32, u32, vp, i64, vp]
+        lib.dg_normal_f32.restype = None
+        _host = lib
+    return _host or None
+
+
 def kv_rows(w: Workload, which: str, tokens, heads=None) -> np.ndarray:
     """Exact float32 values of K or V at global token indices ``tokens`` (and heads).
 
     The cache layout is [sum L, H, Dh] row-major; element (t, h, d) is element
     ``(t * H + h) * Dh + d`` of the stream. Returns [len(tokens), len(heads), Dh].
     """
-    tokens = np.asarray(tokens, dtype=np.int64)
-    heads = np.arange(w.H) if heads is None else np.asarray(heads, dtype=np.int64)
+    tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+    heads = np.ascontiguousarray(np.arange(w.H) if heads is None else heads, dtype=np.int64)
+    if tokens.size * heads.size * w.Dh >= _NATIVE_MIN:
+        lib = _host_lib()
+        if lib is not None:  # the same definition in C (bit-identical, tested), for large slices
+            out = np.empty((tokens.size, heads.size, w.Dh), dtype=np.float32)
+            lib.dg_cache_rows(w.seed, TENSOR_IDS[which], w.H, w.Dh, tokens.ctypes.data, tokens.size,
+                              heads.ctypes.data, heads.size, 1 if w.kv_dtype == "bf16" else 0, out.ctypes.data)
+            return out
     idx = ((tokens[:, None, None] * w.H + heads[None, :, None]) * w.Dh
            + np.arange(w.Dh)[None, None, :])
     x = normal_f32(w.seed, TENSOR_IDS[which], idx.reshape(-1)).reshape(idx.shape)

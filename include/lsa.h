@@ -30,6 +30,9 @@
  *     range, a bounded wait that gave up) set bits of a sticky error word at the
  *     start of the workspace; the kernels then skip the bad item instead of
  *     faulting. lsa_get_device_status reads and clears that word.
+ *   - Per-device facts (SM count, kernel attributes) are looked up on the first
+ *     call made on a device and cached for the life of the process; the library
+ *     is not meant to be used across a cudaDeviceReset.
  *   - Ragged batches: with chunk_offsets != NULL, sequence b owns chunks
  *     [chunk_offsets[b], chunk_offsets[b+1]) of the flattened chunk axis and
  *     tokens [chunk_offsets[b]*C, chunk_offsets[b+1]*C) of the K/V caches.
@@ -253,7 +256,10 @@ LSA_API lsa_status lsa_refresh_resident(const lsa_dims *dims, const void *q_emb,
  *   - It calls no allocation routine of any kind.
  *   - The first call on a device (with that device current) looks up the array's
  *     device address and the device's SM count; make that first call before any
- *     stream capture.
+ *     stream capture. Both are cached per process and per device ordinal for the
+ *     life of the process: after cudaDeviceReset (a new primary context) the cached
+ *     address names an array that no longer exists, so do not use this entry point
+ *     across a device reset.
  *   - All calls on a device share the array, which keeps the last call's contents;
  *     each call clears the device error word it uses. Calls whose kernels overlap
  *     on the GPU race on the array: order them on one stream.

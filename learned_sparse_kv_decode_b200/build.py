@@ -39,8 +39,12 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
            "-o", tmp]
     if verbose:
         print(" ".join(cmd))
-    subprocess.check_call(cmd)
-    os.replace(tmp, LIB)  # atomic: a loader never sees a partial file
+    try:
+        subprocess.check_call(cmd)
+        os.replace(tmp, LIB)  # atomic: a loader never sees a partial file
+    finally:
+        if os.path.exists(tmp):  # a failed compile leaves no temporary behind
+            os.remove(tmp)
     return LIB
 
 

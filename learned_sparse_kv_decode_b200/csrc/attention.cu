@@ -118,7 +118,7 @@ k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
     uint64_t* bars = reinterpret_cast<uint64_t*>(scratch + (kAttnConsumers / LPH) * (kDh + 2));
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kStages);
     __shared__ int s_abort;  // set by a consumer whose bounded wait gave up
-    __shared__ int s_skip[kStages];  // ring slot holds no tokens (kept position >= the sequence's count)
+    __shared__ int s_skip[kStages];  // ring slot holds no tokens (past the sequence's count, or a bad id)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x, hs = blockIdx.y;
@@ -161,7 +161,8 @@ k_attn_split(const uint8_t* __restrict__ q, const uint8_t* __restrict__ K,
                     const int n_b = tab.chunk_off[b + 1] - tab.chunk_off[b];
                     if (id < 0 || id >= n_b) {
                         set_error(err, kErrBadId);
-                        mbar_arrive(full0 + 8 * slot);  // release the slot, contents stale
+                        s_skip[slot] = 1;               // the sequence attends over its valid ids only
+                        mbar_arrive(full0 + 8 * slot);  // release the slot without data
                         continue;
                     }
                     token0 = ((int64_t)tab.chunk_off[b] + id) * tab.C + within;

@@ -141,7 +141,8 @@ __device__ __forceinline__ int la_cta_of(int64_t s, const LaParams& lp) {
 }
 
 // Token row (in the K/V tensor) of box j of global tile s. A box past the sequence's kept
-// tokens (a ragged last tile, C < 64) reloads a kept chunk; the softmax masks its scores.
+// tokens (a ragged last tile, C < 64) reloads a kept chunk, and a box of an out-of-range id
+// loads chunk 0 of the sequence; the softmax masks the scores of both (la_bad_tokens).
 __device__ __forceinline__ int la_box_row(int64_t s, int j, const int32_t* __restrict__ ids,
                                           const SeqTable& tab, const LaParams& lp, uint32_t* err) {
     const LaCursor u = la_cursor(s, tab, lp);
@@ -160,6 +161,24 @@ __device__ __forceinline__ int la_box_row(int64_t s, int j, const int32_t* __res
         id = 0;
     }
     return (tab.chunk_off[u.b] + id) * tab.C + off;
+}
+
+// Tokens of the half tile that holds kept-token positions u0 .. u0 + 63 of run cursor u whose
+// chunk id is out of range, as a 64-bit mask (bit j: position u0 + j). Positions past the kept
+// tokens are left to the caller's count.
+__device__ __forceinline__ uint64_t la_bad_tokens(const LaCursor& u, int u0, const int32_t* __restrict__ ids,
+                                                  const SeqTable& tab) {
+    const int kb = tab.kept_off[u.b + 1] - tab.kept_off[u.b];
+    const int nb = tab.chunk_off[u.b + 1] - tab.chunk_off[u.b];
+    uint64_t bad = 0;
+    const int step = tab.C < la::kHalfTok ? tab.C : la::kHalfTok;  // tokens of one chunk inside the half
+    for (int x = 0; x < la::kHalfTok; x += step) {
+        const int kc = (u0 + x) / tab.C;
+        if (kc >= kb) break;
+        const int32_t id = ids[tab.kept_off[u.b] + kc];
+        if (id < 0 || id >= nb) bad |= (step == 64 ? ~0ull : ((1ull << step) - 1ull)) << x;
+    }
+    return bad;
 }
 
 // ------------------------------------------------------------------ tcgen05 / TMA helpers
@@ -529,6 +548,7 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         const uint32_t o0 = lane_t + kTmemO, o1 = o0 + kDh, o_mine = g ? o1 : o0;
         float* scratch = reinterpret_cast<float*>(la_raw + (sX - raw));  // run-end merge scratch
         LaCursor cur = la_cursor(s0, tab, lp);
+        if (lp.indexed) pdl_wait();  // the chunk ids (read for the bad-id mask) come from the preceding kernel
         float m = -INFINITY, l = 0.f;
         bool dead = false, run_whole = false;
         int run_idx = 0;
@@ -542,6 +562,20 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 run0 = i;
             }
             if ((int)(i & 1) == g) {
+                // valid tokens of this row's half tile, 32 at a time: inside the kept tokens and
+                // not from a chunk whose id is out of range
+                uint32_t vm[2];
+                {
+                    const int u0 = cur.t * kTile + half * kHalfTok;
+                    const int rem = cur.kt - u0;
+                    const uint64_t bad = lp.indexed ? la_bad_tokens(cur, u0, ids, tab) : 0ull;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int lo = hh * 32;
+                        vm[hh] = rem >= lo + 32 ? ~0u : (rem <= lo ? 0u : (1u << (rem - lo)) - 1u);
+                        vm[hh] &= ~(uint32_t)(bad >> lo);
+                    }
+                }
                 // 1. this row's scores of tile i
                 dead = la_wait_warp(dead, sf0 + 8 * (uint32_t)(i % kSBufs), (uint32_t)(i / kSBufs) & 1u, err,
                                     &s_abort);
@@ -549,7 +583,6 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 // this row's 64 scores (tokens half*64 .. half*64+63 of the tile) are read twice from
                 // TMEM, 32 at a time: once for the tile max, once for P (fewer live registers)
                 const uint32_t sbuf = lane_t + (uint32_t)(i % kSBufs) * kTile;
-                const int rem = cur.kt - (cur.t * kTile + half * kHalfTok);  // valid tokens of the row
                 float mt = -INFINITY;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
@@ -567,7 +600,7 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                         float v[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
-                            v[e] = hh * 32 + 8 * j + e < rem ? __uint_as_float(sr[8 * j + e]) : -INFINITY;
+                            v[e] = (vm[hh] >> (8 * j + e)) & 1u ? __uint_as_float(sr[8 * j + e]) : -INFINITY;
                         mx[j] = fmaxf(fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])), fmaxf(fmaxf(v[4], v[5]), fmaxf(v[6], v[7])));
                     }
                     mt = fmaxf(mt, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
@@ -625,10 +658,9 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     for (int q8 = 0; q8 < 4; ++q8) {
                         float p[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int j = hb * 32 + 8 * q8 + e;
-                            p[e] = j < rem ? la_ex2(fmaf(__uint_as_float(sr[8 * q8 + e]), lp.qscale, nm)) : 0.f;
-                        }
+                        for (int e = 0; e < 8; ++e)
+                            p[e] = (vm[hb] >> (8 * q8 + e)) & 1u ? la_ex2(fmaf(__uint_as_float(sr[8 * q8 + e]), lp.qscale, nm))
+                                                                 : 0.f;
                         ps[hb * 4 + q8] = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -704,7 +736,7 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     const int64_t slot = 2 * (int64_t)c + (run_idx == 0 ? 0 : 1);
                     float* dst = whole ? out + (((int64_t)cur.b * lp.Qw + qrow) * lp.H + cur.h) * kDh
                                        : part_o + (slot * lp.Qw + qrow) * kDh;
-                    const float inv = whole ? 1.f / L2 : 1.f;
+                    const float inv = whole ? (L2 > 0.f ? 1.f / L2 : 0.f) : 1.f;  // no valid token: out 0
 #pragma unroll 1
                     for (int cc = 0; cc < kDh / 16; ++cc) {
                         uint32_t a[16], bq[16];
@@ -807,7 +839,7 @@ k_attn_la_merge(const float* __restrict__ part_o, const float* __restrict__ part
         }
         M = Mn;
     }
-    const float inv = 1.f / L;
+    const float inv = L > 0.f ? 1.f / L : 0.f;  // no valid token (every id bad): out 0, lse -inf
     float* dst = out + (((int64_t)b * lp.Qw + q) * lp.H + h) * kDh + lane * 4;
     *reinterpret_cast<float4*>(dst) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     if (lse != nullptr && lane == 0) lse[((int64_t)b * lp.Qw + q) * lp.H + h] = (M + log2f(L)) * la::kLn2;

@@ -18,8 +18,12 @@ def build(force: bool = False) -> str:
     # -ffp-contract=off: every multiply and add rounds on its own, as written.
     cmd = ["gcc", "-O2", "-std=c99", "-ffp-contract=off", "-fno-fast-math", "-shared", "-fPIC",
            SRC, "-o", tmp, "-lm"]
-    subprocess.check_call(cmd)
-    os.replace(tmp, LIB)  # atomic: a loader never sees a partial file
+    try:
+        subprocess.check_call(cmd)
+        os.replace(tmp, LIB)  # atomic: a loader never sees a partial file
+    finally:
+        if os.path.exists(tmp):  # a failed compile leaves no temporary behind
+            os.remove(tmp)
     return LIB
 
 

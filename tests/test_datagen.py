@@ -78,3 +78,27 @@ def test_lookahead_queries_layout_and_storage():
     v = datagen.normal_f32(w.seed, datagen.TENSOR_IDS["q_la"], np.array([idx]))[0]
     assert x[b, j, h, d] == datagen.bf16_bits(np.array([v], np.float32))[0]
     assert datagen.TENSOR_IDS["q_la"] not in [t for k, t in datagen.TENSOR_IDS.items() if k != "q_la"]
+
+
+def test_kv_rows_native_matches_numpy_definition():
+    # the C regenerator of large cache slices against the numpy definition, bit for bit,
+    # for both storage types, unordered tokens and a head subset
+    lib = datagen._host_lib()
+    assert lib is not None, "the host generator must build (gcc)"
+    for kv in ("f32", "bf16"):
+        w = datagen.small_workload(H=16, kv_dtype=kv, seed=9)
+        tokens = np.array([4095, 0, 17, 3000, 63, 64, 2047, 5], dtype=np.int64)
+        heads = np.array([15, 0, 7], dtype=np.int64)
+        saved = datagen._NATIVE_MIN
+        try:
+            datagen._NATIVE_MIN = 0
+            native = datagen.kv_rows(w, "V", tokens, heads)
+            datagen._NATIVE_MIN = 1 << 62
+            ref = datagen.kv_rows(w, "V", tokens, heads)
+        finally:
+            datagen._NATIVE_MIN = saved
+        np.testing.assert_array_equal(native.view(np.uint32), ref.view(np.uint32))
+    idx = np.array([0, 1, 2**40 + 3, 123456789], dtype=np.uint64)
+    out = np.empty(idx.size, dtype=np.float32)
+    lib.dg_normal_f32(3, 4, idx.ctypes.data, idx.size, out.ctypes.data)
+    np.testing.assert_array_equal(out, datagen.normal_f32(3, 4, idx))

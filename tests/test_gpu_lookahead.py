@@ -110,6 +110,28 @@ def test_lookahead_attention_parity(lsa, case):
     _free()
 
 
+@pytest.mark.parametrize("C", [64, 16, 256])
+def test_lookahead_bad_id_reported(lsa, C):
+    # out-of-range ids are reported and masked: each sequence's window attends over its valid
+    # ids only, including the sequences that hold the bad ids; no valid id: out 0, lse -inf
+    w = datagen.small_workload(B=4, N=(4, 6, 9, 3), k=(2, 3, 4, 1), E=64, Q=64, H=2, C=C, kv_dtype="bf16",
+                               emb_dtype="bf16", seed=63)
+    win = Window(w, lsa)
+    ids = np.array([0, 1,  2, -3, 5,  1, 9, 4, 8,  3], dtype=np.int32)
+    valid = [np.array([0, 1]), np.array([2, 5]), np.array([1, 4, 8]), None]
+    lsa.lsa_sparse_decode_attn_lookahead(win.dw.dims, win.q, win.dw.K, win.dw.V, torch.from_numpy(ids).cuda(),
+                                         win.out, win.lse, win.dw.ws)
+    assert lsa.lsa_get_device_status(win.dw.ws) == lsa.LSA_ERR_BAD_ID
+    for b, v in enumerate(valid):
+        if v is None:
+            np.testing.assert_array_equal(win.out[b].cpu().numpy(), 0.0)
+            assert np.isneginf(win.lse[b].cpu().numpy()).all()
+            continue
+        _compare(win, b, v)
+    del win
+    _free()
+
+
 def test_lookahead_resident_equals_indexed(lsa):
     # the same tiles in the same order: the resident form gives bit-identical results
     w = datagen.small_workload(B=2, N=(40, 72), k=(5, 9), C=16, E=64, Q=64, H=4, kv_dtype="bf16",
