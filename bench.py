@@ -35,6 +35,7 @@ sys.path.insert(0, ROOT)
 METRIC = "LSA decode steps/s and achieved HBM GB/s (% roofline) at 128K/500K/1M ctx"
 SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
 
 
 def parse_args():
@@ -309,12 +310,22 @@ class Setup:
 
         self.w = w
         x = datagen.make_inputs(w)
-        self.chunk_emb = dev(x["chunk_emb"], w.emb_dtype)
+        # enough copies of the chunk embeddings (same values, distinct addresses) that the copies
+        # the steps cycle through sum to more than twice the L2: every step's scoring reads them
+        # from HBM, not from what the previous steps left in L2
+        emb = dev(x["chunk_emb"], w.emb_dtype)
+        # (a step that fits in L2 as a whole -- the tiny parity workload -- keeps one copy: its K/V
+        # are L2-resident anyway, and it is reported as launch-bound)
+        n_emb = 1 if w.algorithmic_bytes() < L2_BYTES else -(-2 * L2_BYTES // (emb.numel() * emb.element_size()))
+        self.chunk_embs = [emb] + [emb.clone() for _ in range(n_emb - 1)]
+        self.chunk_emb = emb
         self.q_emb, self.q = [], []
         for r in range(rotations):
             v = datagen.make_query_variant(w, r)
             self.q_emb.append(dev(v["q_emb"], w.emb_dtype))
             self.q.append(dev(v["q"], w.kv_dtype))
+        # one graph per (query set, embedding copy) pair of the cycle
+        self.cycle = max(rotations, n_emb)
         tdt = torch.bfloat16 if w.kv_dtype == "bf16" else torch.float32
         L = int(sum(w.L))
         self.K = torch.empty((L, w.H, w.Dh), dtype=tdt, device="cuda")
@@ -334,8 +345,12 @@ class Setup:
         self.lsa = lsa
         torch.cuda.synchronize()
 
-    def step(self, r: int, stream=None):
-        self.lsa.lsa_decode_step(self.dims, self.q_emb[r], self.chunk_emb, self.q[r], self.K, self.V,
+    def emb(self, i: int):
+        return self.chunk_embs[i % len(self.chunk_embs)]
+
+    def step(self, i: int, stream=None):
+        r = i % len(self.q)
+        self.lsa.lsa_decode_step(self.dims, self.q_emb[r], self.emb(i), self.q[r], self.K, self.V,
                                  self.ids, self.out, self.lse, self.ws, stream)
 
     def capture(self):
@@ -344,14 +359,14 @@ class Setup:
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
-            for r in range(len(self.q)):
-                self.step(r)
+            for i in range(self.cycle):
+                self.step(i)
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
-        for r in range(len(self.q)):
+        for i in range(self.cycle):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                self.step(r)
+                self.step(i)
             self.graphs.append(g)
         torch.cuda.synchronize()
         st = self.lsa.lsa_get_device_status(self.ws)
@@ -360,6 +375,14 @@ class Setup:
 
     def step_bytes(self) -> int:
         return self.w.algorithmic_bytes()
+
+    def emb_bytes(self) -> int:
+        w = self.w
+        return (w.total_chunks + w.B * w.Q) * w.E * w.esize("emb_dtype")
+
+    def kept_kv_bytes(self) -> int:
+        w = self.w
+        return w.total_kept * w.C * w.H * w.Dh * w.esize("kv_dtype") * 2
 
     def attn_bytes(self) -> int:
         w = self.w
@@ -444,6 +467,9 @@ def run_ours(args):
                "gbs_per_gpu": S.step_bytes() * K / (ms / 1e3) / 1e9, "bytes_per_step": S.step_bytes()}
         res["frac_of_measured"] = res["gbs_per_gpu"] / peak
         res["frac_of_spec_8tbs"] = res["gbs_per_gpu"] / SPEC_HBM_GBS
+        # the stages alone: scoring (HBM, embeddings not L2-resident), top-k (latency), the standalone
+        # gather (read + write of the kept K/V)
+        res["kernels"] = kernel_loops(S, min(K, 640), W, world, peak)
         if name in ("1m", "1m-h2"):
             # the pages' own indexer score (FP8 compressed-K, 3 layers x 128 heads) feeding the same step
             res["fp8_indexer_step"] = fp8_step_loop(S, K, W, world)
@@ -463,7 +489,7 @@ def run_ours(args):
             res["step_us"] = {"p10": per[20], "p50": per[100], "p90": per[180], "n": len(per),
                               "note": "each replay timed alone (so each includes one graph-launch gap)"}
             # the dominant kernel alone: split-K attention (+ its merge) over the last step's kept ids
-            r_last = (K - 1) % R
+            r_last = (K - 1) % len(S.q)
             ams = time_loop(lambda i: lsa.lsa_sparse_decode_attn(S.dims, S.q[r_last], S.K, S.V, S.ids, S.out,
                                                                  S.lse, S.ws), K, W, world)
             res["attn_ms"] = ams / K
@@ -514,7 +540,9 @@ def run_ours(args):
                 "parallelism": f"replicas x{world} (independent sequences, no collective)",
                 "storage": {"emb": w.emb_dtype, "kv": w.kv_dtype},
                 "l2": (f"inputs larger than L2: each step streams {head.step_bytes() / 1e9:.3f} GB "
-                       f"(126 MB L2); {R} rotating query sets"),
+                       f"(126 MB L2); {len(head.q)} rotating query sets and {len(head.chunk_embs)} copies of "
+                       f"the chunk embeddings cycled ({len(head.chunk_embs) * head.emb_bytes() / 2**20:.0f} MiB, "
+                       "over twice the L2), so scoring reads them from HBM"),
                 "cuda_graph": True,
             },
             "gbs": hr["gbs_per_gpu"] * world,
@@ -527,6 +555,9 @@ def run_ours(args):
                 "peak": peak,
                 "unit": "GB/s",
                 "frac": attn_gbs / peak,
+                "frac_of_spec_8tbs": attn_gbs / SPEC_HBM_GBS,
+                "peak_note": ("peak = the measured copy bandwidth (read + write); a read-only stream can "
+                              "exceed it, so frac_of_spec_8tbs is given beside it"),
                 "traffic": recorded_traffic(args.workload),
                 "algorithmic_bytes_per_launch": head.attn_bytes(),
                 "launch_ms": hr["attn_ms"],
@@ -548,31 +579,145 @@ def run_ours(args):
     return 0
 
 
+def graph_loop(call, n: int, K: int, W: int, world: int) -> float:
+    """Device time (ms) of one call: `n` consecutive calls call(0..n-1) captured in one CUDA graph,
+    replayed so that K calls are timed (CUDA events, max over ranks). Host launch overhead is out of
+    the timed region; each call still pays its kernel launch gaps on the device."""
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for i in range(n):
+            call(i)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n):
+            call(i)
+    reps = max(1, K // n)
+    ms = time_loop(lambda i: g.replay(), reps, max(1, W // n), world)
+    del g
+    return ms / (reps * n)
+
+
+def kernel_loops(S, K: int, W: int, world: int, peak_gbs: float) -> dict:
+    """Each stage of the step timed alone (graphs of consecutive calls, CUDA events, max over ranks):
+    lsa_score_chunks over the rotating embedding copies (all chunk embeddings + query embeddings
+    from HBM), lsa_topk_select on the step's scores, and lsa_gather_kv of the last step's kept
+    ids into a resident buffer (read + write of the kept K/V)."""
+    import torch
+    w, lsa = S.w, S.lsa
+    R = len(S.q)
+    n_emb = len(S.chunk_embs)
+    scores = torch.empty(w.total_chunks, dtype=torch.float32, device="cuda")
+    n = max(n_emb, 32)
+    ms_s = graph_loop(lambda i: lsa.lsa_score_chunks(S.dims, S.q_emb[i % R], S.emb(i), scores, S.ws), n, K, W, world)
+    ids = torch.empty_like(S.ids)
+    ms_k = graph_loop(lambda i: lsa.lsa_topk_select(S.dims, scores, ids, S.ws), 32, K, W, world)
+    K_res = torch.empty((w.total_kept * w.C, w.H, w.Dh), dtype=S.K.dtype, device="cuda")
+    V_res = torch.empty_like(K_res)
+    ms_g = graph_loop(lambda i: lsa.lsa_gather_kv(S.dims, S.K, S.V, S.ids, K_res, V_res, S.ws), 4, K // 8, W, world)
+    st = lsa.lsa_get_device_status(S.ws)
+    if st != lsa.LSA_OK:
+        raise SystemExit(f"device error in the stage loops: {lsa.string(st)}")
+    del K_res, V_res
+    torch.cuda.empty_cache()
+    t_s, t_k, t_g = ms_s / 1e3, ms_k / 1e3, ms_g / 1e3
+    gb_s = S.emb_bytes() / t_s / 1e9
+    g_bytes = 2 * S.kept_kv_bytes() + w.total_kept * 4
+    gb_g = g_bytes / t_g / 1e9
+    return {
+        "score": {"us": t_s * 1e6, "gbs": gb_s, "frac_of_measured": gb_s / peak_gbs, "bytes": S.emb_bytes(),
+                  "embedding_copies": n_emb},
+        "topk": {"us": t_k * 1e6, "keys": w.total_chunks, "kept": w.total_kept},
+        "gather": {"us": t_g * 1e6, "gbs": gb_g, "frac_of_measured": gb_g / peak_gbs, "bytes": g_bytes,
+                   "note": "lsa_gather_kv: kept K/V read once and written once to a resident buffer"},
+        "note": "each stage alone, back to back in a CUDA graph: a call's time includes one kernel launch gap",
+    }
+
+
 def e2e_loop(S, K: int, W: int, world: int) -> dict:
-    """Steps/s through lsa_decode_step with pinned host buffers: per step H2D of the queries,
-    the step, D2H of the kept ids and the attention output."""
+    """Steps/s through lsa_decode_step with pinned host memory. Every step copies its inputs
+    host -> device (the query embeddings and decode queries, packed in one pinned buffer: one
+    copy) and its results device -> host (attention output and kept ids, packed in one device
+    buffer: one copy). The copies run on two copy streams into double buffers, so the copies of
+    step i overlap the kernels of steps i - 1 and i + 1; events order every buffer reuse. The
+    timed region runs from before the first H2D copy to after the last D2H copy."""
     import torch
     R = len(S.q)
-    hq_emb = [t.cpu().pin_memory() for t in S.q_emb]
-    hq = [t.cpu().pin_memory() for t in S.q]
-    h_out = torch.empty(S.out.shape, dtype=S.out.dtype).pin_memory()
-    h_ids = torch.empty(S.ids.shape, dtype=S.ids.dtype).pin_memory()
-    d_q_emb = torch.empty_like(S.q_emb[0])
-    d_q = torch.empty_like(S.q[0])
+    main = torch.cuda.current_stream()
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def a16(n):
+        return (n + 15) // 16 * 16
+
+    qe0, q0 = S.q_emb[0], S.q[0]
+    nb_qe, nb_q = qe0.numel() * qe0.element_size(), q0.numel() * q0.element_size()
+    off_q = a16(nb_qe)
+    in_bytes = off_q + nb_q
+    h_in = []
+    for r in range(R):
+        h = torch.empty(in_bytes, dtype=torch.uint8).pin_memory()
+        h[:nb_qe].copy_(S.q_emb[r].cpu().contiguous().view(-1).view(torch.uint8))
+        h[off_q:].copy_(S.q[r].cpu().contiguous().view(-1).view(torch.uint8))
+        h_in.append(h)
+    nb_out, nb_ids = S.out.numel() * 4, S.ids.numel() * 4
+    off_ids = a16(nb_out)
+    out_bytes = off_ids + nb_ids
+    d_in = [torch.empty(in_bytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    d_out = [torch.empty(out_bytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    h_out = [torch.empty(out_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
+    qe_v = [d[:nb_qe].view(qe0.dtype).view(qe0.shape) for d in d_in]
+    q_v = [d[off_q:].view(q0.dtype).view(q0.shape) for d in d_in]
+    out_v = [d[:nb_out].view(torch.float32).view(S.out.shape) for d in d_out]
+    ids_v = [d[off_ids:].view(torch.int32) for d in d_out]
+    ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in_ready", "in_free", "out_ready", "out_done")}
 
     def one(i):
-        r = i % R
-        d_q_emb.copy_(hq_emb[r], non_blocking=True)
-        d_q.copy_(hq[r], non_blocking=True)
-        S.lsa.lsa_decode_step(S.dims, d_q_emb, S.chunk_emb, d_q, S.K, S.V, S.ids, S.out, S.lse, S.ws)
-        h_out.copy_(S.out, non_blocking=True)
-        h_ids.copy_(S.ids, non_blocking=True)
+        j, r = i & 1, i % R
+        with torch.cuda.stream(h2d):
+            h2d.wait_event(ev["in_free"][j])
+            d_in[j].copy_(h_in[r], non_blocking=True)
+            ev["in_ready"][j].record(h2d)
+        main.wait_event(ev["in_ready"][j])
+        main.wait_event(ev["out_done"][j])
+        S.lsa.lsa_decode_step(S.dims, qe_v[j], S.emb(i), q_v[j], S.K, S.V, ids_v[j], out_v[j], S.lse, S.ws, main)
+        ev["in_free"][j].record(main)
+        ev["out_ready"][j].record(main)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(ev["out_ready"][j])
+            h_out[j].copy_(d_out[j], non_blocking=True)
+            ev["out_done"][j].record(d2h)
 
-    ms = time_loop(one, K, W, world)
-    bi = d_q_emb.numel() * d_q_emb.element_size() + d_q.numel() * d_q.element_size()
-    bo = h_out.numel() * h_out.element_size() + h_ids.numel() * h_ids.element_size()
-    return {"value": K / (ms / 1e3) * world, "unit": "steps/s", "h2d_bytes_per_step": bi,
-            "d2h_bytes_per_step": bo, "ms_per_step": ms / K}
+    def run(n):
+        h2d.wait_stream(main)
+        d2h.wait_stream(main)
+        for i in range(n):
+            one(i)
+        main.wait_stream(d2h)
+
+    run(W)
+    torch.cuda.synchronize()
+    _barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(main)
+    run(K)
+    t1.record(main)
+    torch.cuda.synchronize()
+    _barrier(world)
+    torch.cuda.synchronize()
+    ms = _max_over_ranks(t0.elapsed_time(t1), world)
+    # the results that came back are the step's own: the last step's ids against the graph step's
+    last = (K - 1) & 1
+    S.step(K - 1)
+    torch.cuda.synchronize()
+    assert torch.equal(ids_v[last].cpu(), S.ids.cpu()), "e2e step returned other ids than the step itself"
+    assert torch.equal(h_out[last][off_ids:].view(torch.int32), S.ids.cpu()), "D2H copy does not hold the ids"
+    return {"value": K / (ms / 1e3) * world, "unit": "steps/s", "h2d_bytes_per_step": in_bytes,
+            "d2h_bytes_per_step": out_bytes, "ms_per_step": ms / K, "copies_per_step": {"h2d": 1, "d2h": 1},
+            "overlap": "double-buffered copy streams"}
 
 
 def lookahead_loop(S, K: int, W: int, world: int, peak_gbs: float) -> dict:
@@ -592,23 +737,24 @@ def lookahead_loop(S, K: int, W: int, world: int, peak_gbs: float) -> dict:
     out = torch.empty((w.B, w.Q, w.H, w.Dh), dtype=torch.float32, device="cuda")
     lse = torch.empty((w.B, w.Q, w.H), dtype=torch.float32, device="cuda")
 
-    def step(r):
-        lsa.lsa_decode_step_lookahead(S.dims, S.q_emb[r], S.chunk_emb, qla[r], S.K, S.V, S.ids, out, lse, S.ws)
+    def step(i):
+        r = i % R
+        lsa.lsa_decode_step_lookahead(S.dims, S.q_emb[r], S.emb(i), qla[r], S.K, S.V, S.ids, out, lse, S.ws)
 
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
-        for r in range(R):
-            step(r)
+        for i in range(S.cycle):
+            step(i)
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
     graphs = []
-    for r in range(R):
+    for i in range(S.cycle):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            step(r)
+            step(i)
         graphs.append(g)
-    ms = time_loop(lambda i: graphs[i % R].replay(), K, W, world)
+    ms = time_loop(lambda i: graphs[i % len(graphs)].replay(), K, W, world)
     r_last = (K - 1) % R
     ams = time_loop(lambda i: lsa.lsa_sparse_decode_attn_lookahead(S.dims, qla[r_last], S.K, S.V, S.ids, out, lse,
                                                                    S.ws), K, W, world)
@@ -635,7 +781,10 @@ def fp8_step_loop(S, K: int, W: int, world: int, layers: int = 3, heads: int = 1
     import datagen
     w, lsa = S.w, S.lsa
     x = datagen.make_indexer_inputs(w, layers, heads)
-    ck = torch.from_numpy(x["compressed_k"]).cuda()
+    ck0 = torch.from_numpy(x["compressed_k"]).cuda()
+    # copies of the compressed keys (same values) cycled so that they sum to more than twice the L2
+    cks = [ck0] + [ck0.clone() for _ in range(max(1, -(-2 * L2_BYTES // ck0.numel())) - 1)]
+    ck = ck0
     q8 = torch.from_numpy(x["q_fp8"]).cuda()
     qs = torch.from_numpy(x["q_scale"]).cuda()
     hw = torch.from_numpy(x["head_w"]).cuda()
@@ -643,24 +792,26 @@ def fp8_step_loop(S, K: int, W: int, world: int, layers: int = 3, heads: int = 1
     dims = lsa.Dims(w.B, 1, lsa.LSA_INDEX_DIM, w.H, w.C, N=w.N[0], k=w.k[0], emb_dtype="bf16",
                     kv_dtype=w.kv_dtype)
 
-    def step(r):
-        lsa.lsa_decode_step_fp8(dims, layers, heads, lsa.LSA_ENSEMBLE_MAX, ck, q8, qs, hw, S.q[r], S.K, S.V,
-                                S.ids, S.out, S.lse, S.ws)
+    n = max(R, len(cks))
+
+    def step(i):
+        lsa.lsa_decode_step_fp8(dims, layers, heads, lsa.LSA_ENSEMBLE_MAX, cks[i % len(cks)], q8, qs, hw,
+                                S.q[i % R], S.K, S.V, S.ids, S.out, S.lse, S.ws)
 
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
-        for r in range(R):
-            step(r)
+        for i in range(n):
+            step(i)
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
     graphs = []
-    for r in range(R):
+    for i in range(n):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            step(r)
+            step(i)
         graphs.append(g)
-    ms = time_loop(lambda i: graphs[i % R].replay(), K, W, world)
+    ms = time_loop(lambda i: graphs[i % n].replay(), K, W, world)
     st = lsa.lsa_get_device_status(S.ws)
     if st != lsa.LSA_OK:
         raise SystemExit(f"device error in the fp8 step: {lsa.string(st)}")
@@ -668,7 +819,8 @@ def fp8_step_loop(S, K: int, W: int, world: int, layers: int = 3, heads: int = 1
     step_bytes = (ck.numel() + q8.numel() + 4 * (qs.numel() + hw.numel())
                   + w.total_kept * w.C * w.H * w.Dh * kv * 2 + w.B * w.H * w.Dh * (kv + 4) + w.total_kept * 4)
     return {"layers": layers, "heads": heads, "steps_per_s": K / (ms / 1e3) * world, "ms_per_step": ms / K,
-            "gbs": step_bytes * K / (ms / 1e3) / 1e9 * world, "bytes_per_step": step_bytes}
+            "gbs": step_bytes * K / (ms / 1e3) / 1e9 * world, "bytes_per_step": step_bytes,
+            "compressed_k_copies": len(cks)}
 
 
 def interval_loop(S, K: int, W: int, world: int, every: int = 64) -> dict:
@@ -684,7 +836,7 @@ def interval_loop(S, K: int, W: int, world: int, every: int = 64) -> dict:
     moved = torch.zeros(w.B, dtype=torch.int32, device="cuda")
 
     def cycle(r):
-        lsa.lsa_refresh_resident(S.dims, S.q_emb[r], S.chunk_emb, S.K, S.V, slots, K_res, V_res, moved, S.ws)
+        lsa.lsa_refresh_resident(S.dims, S.q_emb[r], S.emb(r), S.K, S.V, slots, K_res, V_res, moved, S.ws)
         for i in range(every):
             lsa.lsa_sparse_decode_attn(S.dims, S.q[(r + i) % R], K_res, V_res, None, S.out, S.lse, S.ws)
 
