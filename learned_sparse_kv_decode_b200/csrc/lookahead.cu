@@ -20,33 +20,33 @@
 //    in the kernel parameters.
 //  * Warp 8 (producer) streams each tile's K and V rows from the full cache, through the
 //    kept chunk ids (or from a compact resident buffer), with 3-D TMA tile loads in the
-//    128-byte-swizzled layout the MMAs read: a 2-deep K ring (a K tile is free once its S
-//    has completed) and a 3-deep V ring (free once its O has). No multicast; L2 evict-first.
+//    128-byte-swizzled layout the MMAs read: a 3-deep K ring (a K tile is free once its S has
+//    completed) and a 3-deep V ring (free once its O has). No multicast; L2 evict-first.
 //  * Warp 9 (one thread) issues the MMAs as their inputs arrive (polling, never blocking on
 //    one barrier while another product is ready):
-//      S  = Qd . K^T   M = 128, N = 128, K = 128  bf16 -> fp32 TMEM, 2 buffers
-//      O += P . V      M = 128, N = 128, K = 128  P read from TMEM, V an MN-major smem operand
-//    (A K=16 MMA with N <= 128 costs about the same whatever N, so the tile is as wide as
-//    the S product allows.) Qd holds the window's queries twice (rows 0-63 and 64-127). Rows
-//    0-63 use the scores of the tile's tokens 0-63 and rows 64-127 those of tokens 64-127
-//    (their P is zero over the other half). So each softmax thread owns one (query,
-//    half-tile) row, and all four TMEM lane quarters do work. The MMAs do twice the useful
-//    flops; at 128 flop per K/V byte that still sits under the tensor-pipe roofline.
+//      S  = Q . K^T    M = 64, N = 128, K = 128  bf16 -> fp32 TMEM, 2 buffers
+//      O += P . V      M = 64, N = 128, K = 128  P read from TMEM, V an MN-major smem operand
+//    M = 64 holds the window's queries once. A tcgen05 MMA with N <= 128 takes about the same
+//    time whatever its M (64 or 128) and N, so the tile is as wide as the S product allows;
+//    M = 64 does half the multiply-adds of a 128-row product, and its 16 KiB of queries leave
+//    room for the third K stage.
 //  * Warps 0-3 and 4-7 are two softmax groups that take alternate tiles. Each group has
 //    its own running max m and sum l per row (log2 domain) and its own O accumulator in
-//    TMEM, so two tiles' softmax overlap. A thread reads its 64 scores (tcgen05.ld) and
-//    writes its bf16 P row over the first 64 columns of the same S buffer (tcgen05.st); l
-//    sums the fp32 weights. It rescales its O row only when m grows by more than 8 (2^8);
+//    TMEM, so two tiles' softmax overlap. An M = 64 accumulator keeps row m in TMEM lane
+//    (m % 16) + 32 (m / 16); the 16-lane access shapes give each thread two rows and a quarter
+//    of their columns, so the four threads of a quad share two rows (max by shuffles, each
+//    thread sums the weights of its own tokens). A thread reads its scores (tcgen05.ld) and
+//    writes its bf16 weights over the first 64 columns of the same S buffer (tcgen05.st); l
+//    sums the fp32 weights. A row's O is rescaled only when its m grows by more than 8 (2^8);
 //    a stale max is exact after the final division by l.
 //  * Per S buffer, three mbarriers order the hand-offs: S landed, P written, and the O
 //    product that read P completed. Each completes one phase every two tiles, and the
 //    hand-offs keep every waiter within one phase of it (a parity wait two phases out of
 //    step would pass early).
 //  * At the end of a (b, h) run, group 0 merges its own and group 1's O rows straight from
-//    TMEM (same lanes), then the two half-rows of each query (log-sum-exp). A run wholly
-//    inside the CTA writes out/lse directly. A run split across CTAs writes a partial
-//    (O, m, l) to slot 2c (the CTA's first run) or 2c + 1 (its last run), and
-//    k_attn_la_merge combines them.
+//    TMEM (same lanes, log-sum-exp). A run wholly inside the CTA writes out/lse directly. A
+//    run split across CTAs writes a partial (O, m, l) to slot 2c (the CTA's first run) or
+//    2c + 1 (its last run), and k_attn_la_merge combines them.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -60,18 +60,17 @@ namespace lsa {
 
 namespace la {
 constexpr int kTile = 128;                // kept tokens per tile
-constexpr int kHalfTok = kTile / 2;       // tokens of a tile each MMA row (query copy) attends to
-constexpr int kRows = 128;                // MMA rows: the window's queries, twice
+constexpr int kHalfTok = kTile / 2;       // tokens of a half tile (the bad-id mask is built 64 at a time)
+constexpr int kRows = 64;                 // MMA rows (M = 64): the window's queries
 constexpr int kQmax = 64;                 // window queries per (sequence, head)
-constexpr int kKStages = 2;               // K ring depth (a K tile is free once its S has completed)
+constexpr int kKStages = 3;               // K ring depth (a K tile is free once its S has completed)
 constexpr int kVStages = 3;               // V ring depth (a V tile is free once its O has completed)
 constexpr uint32_t kHalf = kTile * 128;   // a 64-dim half of a K or V tile: 128 rows x 128 B (16 KiB)
 constexpr uint32_t kOperand = 2 * kHalf;  // a K or V tile (32 KiB)
 
-constexpr uint32_t kQHalf = kRows * 128;  // a 64-dim half of Qd (16 KiB)
-constexpr uint32_t kQBytes = 2 * kQHalf;  // Qd (32 KiB)
-constexpr uint32_t kScratch = kQmax * 128 * 4;  // run-end merge: 64 rows x 128 fp32 (32 KiB)
-constexpr uint32_t kSmem = kQBytes + kScratch + (kKStages + kVStages) * kOperand + 1024;  // + alignment slack
+constexpr uint32_t kQHalf = kRows * 128;  // a 64-dim half of the queries (8 KiB)
+constexpr uint32_t kQBytes = 2 * kQHalf;  // the queries (16 KiB)
+constexpr uint32_t kSmem = kQBytes + (kKStages + kVStages) * kOperand + 1024;  // + alignment slack
 constexpr int kThreads = 320;             // warps 0-7 softmax (two groups of 4), 8 producer, 9 MMA
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
@@ -82,7 +81,7 @@ constexpr float kRescale = 8.0f;          // lazy-rescale threshold (log2 units)
 constexpr int kMaxCtas = 256;             // CTAs of one launch (one per SM)
 constexpr int kRunCost = 4;               // extra cost of a run start in the tile split, in tiles (measured)
 constexpr float kLn2 = 0.69314718055994531f;
-static_assert(kQBytes % 1024 == 0 && kScratch % 1024 == 0 && kOperand % 1024 == 0, "1 KiB swizzle atoms");
+static_assert(kQBytes % 1024 == 0 && kOperand % 1024 == 0, "1 KiB swizzle atoms");
 static_assert(kTmemO + 2 * 128 == kTmemCols, "TMEM: S buffers then two O accumulators");
 
 }  // namespace la
@@ -227,10 +226,22 @@ __device__ __forceinline__ void la_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void la_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+// The M = 64 accumulators (S, O) and the P operand hold row m in TMEM lane (m % 16) + 32 (m / 16):
+// lanes 0-15 of each warp's 32-lane quarter. The 16-lane access shapes spread those 16 lanes over
+// the warp's 32 threads; for thread t of the warp, per 8-column (.16x256b) or 4-column (.16x128b)
+// block j of the access:
+//   .16x256b: regs 4j, 4j+1 = lane t/4,     columns 8j + 2(t%4), 8j + 2(t%4) + 1
+//             regs 4j+2, 4j+3 = lane t/4 + 8, the same columns
+//   .16x128b: reg 2j = lane t/4, column 4j + t%4;  reg 2j+1 = lane t/4 + 8, the same column
+// So a thread holds two rows (t/4 and t/4 + 8 of its quarter) and, of a 128-column row, the 32
+// columns 8j + 2(t%4) + {0, 1}; the four threads of a quad (t/4 equal) share their two rows. Its two
+// bf16 weights of block j (tokens 8j + 2(t%4) + {0, 1}) pack into P column 4j + t%4: exactly what
+// .16x128b stores for it.
+
+// 64 columns (8 blocks) of this thread's two rows, .16x256b.
+__device__ __forceinline__ void la_ld256x8(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
         "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
@@ -240,18 +251,21 @@ __device__ __forceinline__ void la_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 
-// 16 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void la_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+__device__ __forceinline__ void la_st256x8(uint32_t taddr, const uint32_t (&r)[32]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
+        "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
 }
 
-__device__ __forceinline__ void la_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+// 32 columns (8 blocks of 4) of this thread's two rows, .16x128b.
+__device__ __forceinline__ void la_st128x8(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+        "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
             taddr),
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
         "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
@@ -334,13 +348,12 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ float2 s_ml1[kRows];  // group 1's (m, l) per row, at a run end
-    __shared__ float2 s_mlh[kQmax];  // merged (m, l) of rows 64..127, at a run end
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x;
     const uint32_t raw = smem_u32(la_raw);
     const uint32_t sQ = (raw + 1023u) & ~1023u;
-    const uint32_t sX = sQ + kQBytes, sK = sX + kScratch, sV = sK + kKStages * kOperand;
+    const uint32_t sK = sQ + kQBytes, sV = sK + kKStages * kOperand;
     const uint32_t kf0 = smem_u32(bar_kf), ke0 = smem_u32(bar_ke), vf0 = smem_u32(bar_vf), ve0 = smem_u32(bar_ve);
     const uint32_t sf0 = smem_u32(bar_sf), pf0 = smem_u32(bar_pf), sx0 = smem_u32(bar_sx);
     const uint32_t qf = smem_u32(&bar_qf), qe = smem_u32(&bar_qe), endb = smem_u32(&bar_end);
@@ -413,9 +426,7 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                             if (qloads > 0 && !mbar_wait(qe, (uint32_t)(qloads - 1) & 1u, err)) dead = true;
                             if (!dead) {
                                 mbar_arrive_expect_tx(qf, kQBytes);
-                                for (int d = 0; d < 2; ++d)
-                                    for (int rr = 0; rr < 2; ++rr)
-                                        la_tma4(sQ + d * kQHalf + rr * (kQHalf / 2), &tmQ, 64 * d, cur.h, 0, cur.b, qf);
+                                for (int d = 0; d < 2; ++d) la_tma4(sQ + d * kQHalf, &tmQ, 64 * d, cur.h, 0, cur.b, qf);
                                 ++qloads;
                             }
                         }
@@ -542,83 +553,108 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         }
     } else {
         // ------------------------------------------------ softmax: two groups of 128 threads take
-        // alternate tiles; thread r of a group owns TMEM lane r and its group's O row r
-        const int g = warp >> 2, r = tid & 127, half = r >> 6, qrow = r & 63;
-        const uint32_t lane_t = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        // alternate tiles. Warp w of a group reads TMEM lane quarter w % 4, which holds rows
+        // 16 (w % 4) .. 16 (w % 4) + 15 of the M = 64 accumulators; thread t of the warp owns rows
+        // r0 = 16 (w % 4) + t/4 and r1 = r0 + 8 (window queries) and, of each 128-token tile, the
+        // tokens 8j + 2 (t % 4) + {0, 1}, j = 0..15. The four threads of a quad share their rows:
+        // the running max is the quad's, each thread sums the weights of its own tokens.
+        const int g = warp >> 2, sp = warp & 3, cq = lane & 3;
+        const int r0 = sp * 16 + (lane >> 2), r1 = r0 + 8;
+        const uint32_t lane_t = tmem + ((uint32_t)(sp * 32) << 16);
         const uint32_t o0 = lane_t + kTmemO, o1 = o0 + kDh, o_mine = g ? o1 : o0;
-        float* scratch = reinterpret_cast<float*>(la_raw + (sX - raw));  // run-end merge scratch
         LaCursor cur = la_cursor(s0, tab, lp);
         if (lp.indexed) pdl_wait();  // the chunk ids (read for the bad-id mask) come from the preceding kernel
-        float m = -INFINITY, l = 0.f;
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
         bool dead = false, run_whole = false;
         int run_idx = 0;
         int run0 = 0;
         for (int i = 0; i < n; ++i) {
             const bool last = (i == n - 1) || cur.t == cur.nt - 1;
             if (i == 0 || cur.t == 0) {
-                m = -INFINITY;
-                l = 0.f;
+                m0 = m1 = -INFINITY;
+                l0 = l1 = 0.f;
                 run_whole = cur.t == 0;
                 run0 = i;
             }
             if ((int)(i & 1) == g) {
-                // valid tokens of this row's half tile, 32 at a time: inside the kept tokens and
-                // not from a chunk whose id is out of range
-                uint32_t vm[2];
+                // valid tokens among this thread's 32 (bit 2j + e: token 8j + 2 cq + e of the tile):
+                // inside the kept tokens and not from a chunk whose id is out of range
+                uint32_t vm = 0xFFFFFFFFu;
                 {
-                    const int u0 = cur.t * kTile + half * kHalfTok;
+                    const int u0 = cur.t * kTile;
                     const int rem = cur.kt - u0;
-                    const uint64_t bad = lp.indexed ? la_bad_tokens(cur, u0, ids, tab) : 0ull;
+                    uint64_t bad0 = 0ull, bad1 = 0ull;
+                    if (lp.indexed) {
+                        bad0 = la_bad_tokens(cur, u0, ids, tab);
+                        if (rem > kHalfTok) bad1 = la_bad_tokens(cur, u0 + kHalfTok, ids, tab);
+                    }
+                    if (rem < kTile || (bad0 | bad1) != 0ull) {
+                        vm = 0u;
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int lo = hh * 32;
-                        vm[hh] = rem >= lo + 32 ? ~0u : (rem <= lo ? 0u : (1u << (rem - lo)) - 1u);
-                        vm[hh] &= ~(uint32_t)(bad >> lo);
+                        for (int j = 0; j < 16; ++j) {
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int tok = 8 * j + 2 * cq + e;
+                                const uint64_t bw = tok < kHalfTok ? bad0 : bad1;
+                                if (tok < rem && !((bw >> (tok & 63)) & 1ull)) vm |= 1u << (2 * j + e);
+                            }
+                        }
                     }
                 }
-                // 1. this row's scores of tile i
+                // 1. the scores of tile i, 64 columns at a time; read twice from TMEM (once for the
+                // tile max, once for P) to keep fewer registers live
                 dead = la_wait_warp(dead, sf0 + 8 * (uint32_t)(i % kSBufs), (uint32_t)(i / kSBufs) & 1u, err,
                                     &s_abort);
                 la_fence_after();
-                // this row's 64 scores (tokens half*64 .. half*64+63 of the tile) are read twice from
-                // TMEM, 32 at a time: once for the tile max, once for P (fewer live registers)
                 const uint32_t sbuf = lane_t + (uint32_t)(i % kSBufs) * kTile;
-                float mt = -INFINITY;
+                float mt0 = -INFINITY, mt1 = -INFINITY;
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
+                for (int w = 0; w < 2; ++w) {
                     uint32_t sr[32];
                     if (!dead) {
-                        la_ld32(sbuf + (uint32_t)(half * kHalfTok + hh * 32), sr);
+                        la_ld256x8(sbuf + (uint32_t)(w * 64), sr);
                         la_wait_ld();
                     } else {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) sr[j] = 0u;
                     }
-                    float mx[4];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        float v[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            v[e] = (vm[hh] >> (8 * j + e)) & 1u ? __uint_as_float(sr[8 * j + e]) : -INFINITY;
-                        mx[j] = fmaxf(fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])), fmaxf(fmaxf(v[4], v[5]), fmaxf(v[6], v[7])));
+                    for (int j = 0; j < 8; ++j) {
+                        const int bit = 2 * (8 * w + j);
+                        const bool v0 = (vm >> bit) & 1u, v1 = (vm >> (bit + 1)) & 1u;
+                        mt0 = fmaxf(mt0, fmaxf(v0 ? __uint_as_float(sr[4 * j]) : -INFINITY,
+                                               v1 ? __uint_as_float(sr[4 * j + 1]) : -INFINITY));
+                        mt1 = fmaxf(mt1, fmaxf(v0 ? __uint_as_float(sr[4 * j + 2]) : -INFINITY,
+                                               v1 ? __uint_as_float(sr[4 * j + 3]) : -INFINITY));
                     }
-                    mt = fmaxf(mt, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
                 }
-                mt *= lp.qscale;
-                // 2. running max (log2 domain); O is rescaled only when the max grows past 2^8
-                const float mn = fmaxf(m, mt);
-                float alpha = 1.f;
+                mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, 1));
+                mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, 2));
+                mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, 1));
+                mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, 2));
+                mt0 *= lp.qscale;
+                mt1 *= lp.qscale;
+                // 2. running max (log2 domain); a row's O is rescaled only when its max grows past 2^8
+                const float mn0 = fmaxf(m0, mt0), mn1 = fmaxf(m1, mt1);
+                float a0 = 1.f, a1 = 1.f;
                 bool need = false;
                 if (i - run0 < 2) {
-                    m = mn;  // this group's first tile of the run: O starts afresh
-                } else if (mn > m + kRescale) {
-                    need = true;
-                    alpha = la_ex2(m - mn);
-                    m = mn;
+                    m0 = mn0;  // this group's first tile of the run: O starts afresh
+                    m1 = mn1;
+                } else {
+                    if (mn0 > m0 + kRescale) {
+                        need = true;
+                        a0 = la_ex2(m0 - mn0);
+                        m0 = mn0;
+                    }
+                    if (mn1 > m1 + kRescale) {
+                        need = true;
+                        a1 = la_ex2(m1 - mn1);
+                        m1 = mn1;
+                    }
                 }
                 if (__any_sync(0xffffffffu, need)) {
-                    // the group's previous O product (tile i - 2) has finished: its O row is stable.
+                    // the group's previous O product (tile i - 2) has finished: its O rows are stable.
                     // (Waited on the per-buffer barrier: S(i) has landed, so O(i - 4) is done and the
                     // phase awaited is the pending one or the last completed, never two ahead.)
                     dead = la_wait_warp(dead, sx0 + 8 * (uint32_t)((i - 2) % kSBufs), (uint32_t)((i - 2) / kSBufs) & 1u,
@@ -626,28 +662,35 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     la_fence_after();
                     if (!dead) {
 #pragma unroll 1
-                        for (int cc = 0; cc < kDh / 16; ++cc) {
-                            uint32_t o[16];
-                            la_ld16(o_mine + (uint32_t)cc * 16, o);
+                        for (int w = 0; w < 2; ++w) {
+                            uint32_t o[32];
+                            la_ld256x8(o_mine + (uint32_t)(w * 64), o);
                             la_wait_ld();
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                            la_st16(o_mine + (uint32_t)cc * 16, o);
+                            for (int j = 0; j < 8; ++j) {
+                                o[4 * j] = __float_as_uint(__uint_as_float(o[4 * j]) * a0);
+                                o[4 * j + 1] = __float_as_uint(__uint_as_float(o[4 * j + 1]) * a0);
+                                o[4 * j + 2] = __float_as_uint(__uint_as_float(o[4 * j + 2]) * a1);
+                                o[4 * j + 3] = __float_as_uint(__uint_as_float(o[4 * j + 3]) * a1);
+                            }
+                            la_st256x8(o_mine + (uint32_t)(w * 64), o);
                         }
                         la_wait_st();
                     }
-                    l *= alpha;
+                    l0 *= a0;
+                    l1 *= a1;
                 }
-                // 3. P = 2^(s*c - m) in bf16 pairs over the first 64 columns of this S buffer (its
-                // scores are in registers): the row's 128 tokens, this half's 64 real and the
-                // other half's zero. l sums the fp32 weights.
-                const float nm = m == -INFINITY ? 0.f : -m;  // all masked so far: every p is 2^-inf = 0
-                float ps[8];
+                // 3. P = 2^(s c - m) as bf16 pairs over the first 64 columns of this S buffer: the
+                // pair of tokens 64w + 8j + 2cq + {0, 1} goes to column 32w + 4j + cq, whose scores
+                // (tokens 64w' with w' <= w) have all been read already. l sums the fp32 weights.
+                const float nm0 = m0 == -INFINITY ? 0.f : -m0;  // all masked so far: every p is 0
+                const float nm1 = m1 == -INFINITY ? 0.f : -m1;
+                float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
-                for (int hb = 0; hb < 2; ++hb) {  // 32 tokens (16 columns of P) at a time
+                for (int w = 0; w < 2; ++w) {
                     uint32_t sr[32];
                     if (!dead) {
-                        la_ld32(sbuf + (uint32_t)(half * kHalfTok + hb * 32), sr);
+                        la_ld256x8(sbuf + (uint32_t)(w * 64), sr);
                         la_wait_ld();
                     } else {
 #pragma unroll
@@ -655,121 +698,106 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     }
                     uint32_t pk[16];
 #pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8) {
-                        float p[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            p[e] = (vm[hb] >> (8 * q8 + e)) & 1u ? la_ex2(fmaf(__uint_as_float(sr[8 * q8 + e]), lp.qscale, nm))
-                                                                 : 0.f;
-                        ps[hb * 4 + q8] = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const __nv_bfloat162 h2 = __floats2bfloat162_rn(p[2 * e], p[2 * e + 1]);
-                            pk[q8 * 4 + e] = *reinterpret_cast<const uint32_t*>(&h2);
-                        }
+                    for (int j = 0; j < 8; ++j) {
+                        const int bit = 2 * (8 * w + j);
+                        const bool v0 = (vm >> bit) & 1u, v1 = (vm >> (bit + 1)) & 1u;
+                        const float p00 = v0 ? la_ex2(fmaf(__uint_as_float(sr[4 * j]), lp.qscale, nm0)) : 0.f;
+                        const float p01 = v1 ? la_ex2(fmaf(__uint_as_float(sr[4 * j + 1]), lp.qscale, nm0)) : 0.f;
+                        const float p10 = v0 ? la_ex2(fmaf(__uint_as_float(sr[4 * j + 2]), lp.qscale, nm1)) : 0.f;
+                        const float p11 = v1 ? la_ex2(fmaf(__uint_as_float(sr[4 * j + 3]), lp.qscale, nm1)) : 0.f;
+                        ps0 += p00 + p01;
+                        ps1 += p10 + p11;
+                        const __nv_bfloat162 h0 = __floats2bfloat162_rn(p00, p01);
+                        const __nv_bfloat162 h1 = __floats2bfloat162_rn(p10, p11);
+                        pk[2 * j] = *reinterpret_cast<const uint32_t*>(&h0);
+                        pk[2 * j + 1] = *reinterpret_cast<const uint32_t*>(&h1);
                     }
-                    // P columns half*32 + hb*16 .. +15 hold scores this row has already read
-                    if (!dead) la_st16(sbuf + (uint32_t)(half * 32 + hb * 16), pk);
+                    if (!dead) la_st128x8(sbuf + (uint32_t)(w * 32), pk);
                 }
-                l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-                if (!dead) {
-                    uint32_t zero[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) zero[j] = 0u;
-                    la_st16(sbuf + (uint32_t)((1 - half) * 32), zero);
-                    la_st16(sbuf + (uint32_t)((1 - half) * 32 + 16), zero);
-                    la_wait_st();
-                }
+                l0 += ps0;
+                l1 += ps1;
+                if (!dead) la_wait_st();
                 la_fence_before();
                 mbar_arrive(pf0 + 8 * (uint32_t)(i % kSBufs));
             }
 
-            // 4. end of this CTA's part of run (b, h): merge the two groups and the two half-rows,
-            // then write out (whole run) or a partial (run split across CTAs)
+            // 4. end of this CTA's part of run (b, h): merge the two groups' rows (same TMEM lanes,
+            // different columns), then write out (whole run) or a partial (run split across CTAs)
             if (last) {
                 const int jl = ((i & 1) == g) ? i : i - 1;  // this group's last tile of the run
                 if (jl >= run0)
                     dead = la_wait_warp(dead, sx0 + 8 * (uint32_t)(jl % kSBufs), (uint32_t)(jl / kSBufs) & 1u, err,
                                         &s_abort);
+                // each row's sum: the quad's four parts
+                float L0 = l0 + __shfl_xor_sync(0xffffffffu, l0, 1);
+                L0 += __shfl_xor_sync(0xffffffffu, L0, 2);
+                float L1 = l1 + __shfl_xor_sync(0xffffffffu, l1, 1);
+                L1 += __shfl_xor_sync(0xffffffffu, L1, 2);
+                if (g == 1 && cq == 0) {
+                    s_ml1[r0] = make_float2(m0, L0);
+                    s_ml1[r1] = make_float2(m1, L1);
+                }
+                la_fence_before();
+                la_softmax_sync();  // group 1's last O has completed and its (m, l) are in s_ml1
                 la_fence_after();
-                if (g == 1) s_ml1[r] = make_float2(m, l);
-                la_softmax_sync();
-                float M = m, L = l, w0 = 0.f, w1 = 0.f;
                 if (g == 0) {
-                    const float2 b1 = s_ml1[r];
-                    M = fmaxf(m, b1.x);
-                    w0 = m == -INFINITY ? 0.f : la_ex2(m - M);
-                    w1 = b1.x == -INFINITY ? 0.f : la_ex2(b1.x - M);
-                    L = w0 * l + w1 * b1.y;
-                    if (half == 1) {  // rows 64..127: both groups' O rows into the scratch
-                        s_mlh[qrow] = make_float2(M, L);
-#pragma unroll 1
-                        for (int cc = 0; cc < kDh / 16; ++cc) {
-                            uint32_t a[16], bq[16];
-                            if (!dead) {
-                                la_ld16(o0 + (uint32_t)cc * 16, a);
-                                la_ld16(o1 + (uint32_t)cc * 16, bq);
-                                la_wait_ld();
-                            }
-#pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                float v = 0.f;
-                                if (!dead) {
-                                    v = w0 != 0.f ? w0 * __uint_as_float(a[j]) : 0.f;
-                                    if (w1 != 0.f) v = fmaf(w1, __uint_as_float(bq[j]), v);
-                                }
-                                scratch[(cc * 16 + j) * kQmax + qrow] = v;
-                            }
-                        }
-                    }
-                }
-                la_softmax_sync();
-                if (g == 0 && half == 0) {
-                    const float2 hb = s_mlh[qrow];
-                    const float M2 = fmaxf(M, hb.x);
-                    const float wa = M == -INFINITY ? 0.f : la_ex2(M - M2);
-                    const float wb = hb.x == -INFINITY ? 0.f : la_ex2(hb.x - M2);
-                    const float L2 = wa * L + wb * hb.y;
-                    const float f0 = wa * w0, f1 = wa * w1;
+                    const float2 b0 = s_ml1[r0], b1 = s_ml1[r1];
+                    const float M0 = fmaxf(m0, b0.x), M1 = fmaxf(m1, b1.x);
+                    // a group that took no tile of the run has m = -inf: weight 0, its O is not read
+                    const float w00 = m0 == -INFINITY ? 0.f : la_ex2(m0 - M0);
+                    const float w01 = b0.x == -INFINITY ? 0.f : la_ex2(b0.x - M0);
+                    const float w10 = m1 == -INFINITY ? 0.f : la_ex2(m1 - M1);
+                    const float w11 = b1.x == -INFINITY ? 0.f : la_ex2(b1.x - M1);
+                    const float LL0 = w00 * L0 + w01 * b0.y, LL1 = w10 * L1 + w11 * b1.y;
                     const bool whole = run_whole && cur.t == cur.nt - 1;
-                    const bool wr = qrow < lp.Qw && !dead;
+                    const bool wr0 = r0 < lp.Qw && !dead, wr1 = r1 < lp.Qw && !dead;
                     const int64_t slot = 2 * (int64_t)c + (run_idx == 0 ? 0 : 1);
-                    float* dst = whole ? out + (((int64_t)cur.b * lp.Qw + qrow) * lp.H + cur.h) * kDh
-                                       : part_o + (slot * lp.Qw + qrow) * kDh;
-                    const float inv = whole ? (L2 > 0.f ? 1.f / L2 : 0.f) : 1.f;  // no valid token: out 0
+                    float* dst0 = whole ? out + (((int64_t)cur.b * lp.Qw + r0) * lp.H + cur.h) * kDh
+                                        : part_o + (slot * lp.Qw + r0) * kDh;
+                    float* dst1 = whole ? out + (((int64_t)cur.b * lp.Qw + r1) * lp.H + cur.h) * kDh
+                                        : part_o + (slot * lp.Qw + r1) * kDh;
+                    // no valid token at all (every id bad): out 0, lse -inf
+                    const float inv0 = whole ? (LL0 > 0.f ? 1.f / LL0 : 0.f) : 1.f;
+                    const float inv1 = whole ? (LL1 > 0.f ? 1.f / LL1 : 0.f) : 1.f;
 #pragma unroll 1
-                    for (int cc = 0; cc < kDh / 16; ++cc) {
-                        uint32_t a[16], bq[16];
+                    for (int w = 0; w < 2; ++w) {
+                        uint32_t oa[32], ob[32];
                         if (!dead) {
-                            la_ld16(o0 + (uint32_t)cc * 16, a);
-                            la_ld16(o1 + (uint32_t)cc * 16, bq);
+                            la_ld256x8(o0 + (uint32_t)(w * 64), oa);
+                            la_ld256x8(o1 + (uint32_t)(w * 64), ob);
                             la_wait_ld();
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) oa[j] = ob[j] = 0u;
                         }
-                        if (wr) {
 #pragma unroll
-                            for (int j = 0; j < 16; j += 4) {
-                                float v[4];
+                        for (int j = 0; j < 8; ++j) {
+                            const int col = 64 * w + 8 * j + 2 * cq;
+                            float x[4];
 #pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    float x = wb != 0.f ? wb * scratch[(cc * 16 + j + e) * kQmax + qrow] : 0.f;
-                                    if (f0 != 0.f) x = fmaf(f0, __uint_as_float(a[j + e]), x);
-                                    if (f1 != 0.f) x = fmaf(f1, __uint_as_float(bq[j + e]), x);
-                                    v[e] = x * inv;
-                                }
-                                *reinterpret_cast<float4*>(dst + cc * 16 + j) = make_float4(v[0], v[1], v[2], v[3]);
+                            for (int e = 0; e < 4; ++e) {
+                                const float wa = e < 2 ? w00 : w10, wb = e < 2 ? w01 : w11;
+                                float v = wa != 0.f ? wa * __uint_as_float(oa[4 * j + e]) : 0.f;
+                                if (wb != 0.f) v = fmaf(wb, __uint_as_float(ob[4 * j + e]), v);
+                                x[e] = v * (e < 2 ? inv0 : inv1);
                             }
+                            if (wr0) *reinterpret_cast<float2*>(dst0 + col) = make_float2(x[0], x[1]);
+                            if (wr1) *reinterpret_cast<float2*>(dst1 + col) = make_float2(x[2], x[3]);
                         }
                     }
-                    if (wr) {
+                    if (cq == 0) {
                         if (whole) {
-                            if (lse != nullptr)
-                                lse[((int64_t)cur.b * lp.Qw + qrow) * lp.H + cur.h] = (M2 + log2f(L2)) * kLn2;
+                            if (lse != nullptr) {
+                                if (wr0) lse[((int64_t)cur.b * lp.Qw + r0) * lp.H + cur.h] = (M0 + log2f(LL0)) * kLn2;
+                                if (wr1) lse[((int64_t)cur.b * lp.Qw + r1) * lp.H + cur.h] = (M1 + log2f(LL1)) * kLn2;
+                            }
                         } else {
-                            *reinterpret_cast<float2*>(part_ml + (slot * lp.Qw + qrow) * 2) = make_float2(M2, L2);
+                            if (wr0) *reinterpret_cast<float2*>(part_ml + (slot * lp.Qw + r0) * 2) = make_float2(M0, LL0);
+                            if (wr1) *reinterpret_cast<float2*>(part_ml + (slot * lp.Qw + r1) * 2) = make_float2(M1, LL1);
                         }
                     }
                 }
-                la_softmax_sync();  // the scratch is read before the next P tiles are written
+                la_softmax_sync();  // s_ml1 is read before a later run end writes it again
                 ++run_idx;
             }
             la_next(cur, tab, lp);
