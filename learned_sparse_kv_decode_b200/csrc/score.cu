@@ -9,10 +9,14 @@
 //
 //   scores[i] = max_{j < Q} sum_e q_emb[b][j][e] * chunk_emb[i][e]      (fp32 accumulate)
 //
-// Two kernels:
-//  * k_score_stream - Q small / fp32: an HBM-bound stream over the chunk
-//    embeddings with 128-bit loads, the query held in registers, and a warp
-//    shuffle reduction per row.
+// Kernels:
+//  * k_score_bulk   - Q = 1, rows of at most 512 bytes: an HBM-bound stream over the
+//    chunk embeddings staged into shared memory by 1-D bulk copies (TMA engine),
+//    read back with 128-bit shared loads, the query piece held in registers, and a
+//    warp shuffle reduction per row.
+//  * k_score_stream - the other CUDA-core cases (Q > 1 without the tensor-core
+//    path, longer rows): 128-bit streaming global loads, the queries in shared
+//    memory.
 //  * k_score_umma   - Q > 1 with bf16 embeddings: a tcgen05 tensor-core GEMM,
 //    D[128 x Qp] = A[128 chunks x E] * B[Qp queries x E]^T accumulated in TMEM,
 //    followed by a per-row max in the epilogue (tcgen05.ld).
@@ -163,6 +167,102 @@ k_score_stream(const uint8_t* __restrict__ q_emb, const uint8_t* __restrict__ em
             for (int u = 0; u < kScoreUnroll; ++u) {
                 const int row = row0 + u * step;
                 if (row < r1) out[row] = best[u];
+            }
+        }
+    }
+}
+
+// ============================================================== TMA-staged stream (Q = 1)
+// One CTA per slab of up to kScoreSlabBytes of consecutive rows of one sequence. Thread 0 issues
+// the slab as kScoreStages 1-D bulk copies (TMA engine, L2 evict-first), each completing on its
+// own mbarrier, all in flight at once. Once they have landed the warps read the rows back with
+// 128-bit shared loads: P lanes per row (one 16-byte piece each) hold the query's matching piece
+// in registers, kScoreUnroll rows at a time, and a shuffle reduction finishes each row. Rows of at most 512 bytes (every workload
+// here); longer rows, and Q > 1 on the CUDA cores, take k_score_stream.
+constexpr int kScoreStages = 4;
+constexpr int kScoreSlabBytes = 32768;
+
+template <bool BF16>
+__global__ void __launch_bounds__(kScoreThreads)
+k_score_bulk(const uint8_t* __restrict__ q_emb, const uint8_t* __restrict__ emb, float* __restrict__ scores,
+             const SeqTable tab, int E, int rows_per_cta, uint32_t* err) {
+    extern __shared__ __align__(128) uint8_t slab[];
+    __shared__ __align__(8) uint64_t bars[kScoreStages];
+    constexpr int ES = BF16 ? 2 : 4;
+    constexpr int VEC = 16 / ES;
+    const int b = blockIdx.y;
+    const int n_b = tab.chunk_off[b + 1] - tab.chunk_off[b];
+    const int r0 = blockIdx.x * rows_per_cta;
+    pdl_trigger();
+    if (r0 >= n_b) return;
+    const int rows = min(n_b - r0, rows_per_cta);
+    const uint32_t row_bytes = (uint32_t)E * ES;
+    const int rps = (rows + kScoreStages - 1) / kScoreStages;  // rows per piece
+    const uint32_t bar0 = smem_u32(bars);
+    const uint32_t sbase = smem_u32(slab);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kScoreStages; ++i) mbar_init(bar0 + 8 * i, 1);
+        fence_mbar_init();
+        const uint64_t pol = policy_evict_first();
+        const uint8_t* src = emb + ((size_t)tab.chunk_off[b] + r0) * row_bytes;
+        for (int i = 0; i < kScoreStages; ++i) {
+            const int a = i * rps, e = min(rows, a + rps);
+            if (a >= e) break;
+            const uint32_t bytes = (uint32_t)(e - a) * row_bytes;
+            mbar_arrive_expect_tx(bar0 + 8 * i, bytes);
+            bulk_g2s(sbase + (uint32_t)a * row_bytes, src + (size_t)a * row_bytes, bytes, bar0 + 8 * i, pol);
+        }
+    }
+
+    const int P = E / VEC;  // 16-byte pieces per row (<= 32)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int RPW = 32 / P;  // rows per warp step
+    const int sub = lane / P, li = lane % P;
+    const int step = (kScoreThreads / 32) * RPW;
+    float qv[8];
+    {
+        const uint8_t* qp = q_emb + ((size_t)b * E + (size_t)li * VEC) * ES;
+        const uint4 t = *reinterpret_cast<const uint4*>(qp);
+        float x[8];
+        unpack16<BF16>(t, x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) qv[e] = x[e];
+    }
+    __syncthreads();  // the barriers are initialised before anyone waits on them
+    // every piece is waited for (bounded), even after a wait gave up: no copy is in flight at exit
+    bool ok = true;
+    for (int i = 0; i < kScoreStages && i * rps < rows; ++i) {
+        const bool landed = mbar_wait(bar0 + 8 * i, 0u, err);
+        ok = ok && landed;
+    }
+    float* out = scores + tab.chunk_off[b] + r0;
+    // kScoreUnroll rows per warp and iteration, independent until their stores; the loop bound is
+    // warp-uniform (every lane joins the shuffles) and rows past the slab are masked
+    for (int wrow = warp * RPW; wrow < rows; wrow += step * kScoreUnroll) {
+        const int row0 = wrow + sub;
+        float acc[kScoreUnroll];
+#pragma unroll
+        for (int u = 0; u < kScoreUnroll; ++u) {
+            const int row = row0 + u * step;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (row < rows && ok)
+                asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                             : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                             : "r"(sbase + (uint32_t)row * row_bytes + (uint32_t)li * 16));
+            float x[8];
+            unpack16<BF16>(v, x);
+            acc[u] = 0.f;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[u] = fmaf(qv[e], x[e], acc[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kScoreUnroll; ++u)
+            for (int off = P >> 1; off > 0; off >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], off);
+        if (li == 0 && ok) {
+#pragma unroll
+            for (int u = 0; u < kScoreUnroll; ++u) {
+                const int row = row0 + u * step;
+                if (row < rows) out[row] = acc[u];
             }
         }
     }
@@ -501,6 +601,8 @@ cudaError_t score_init_attrs() {
     if (e == cudaSuccess) e = set_smem_attrs(k_score_umma_sw, (int)score_umma_sw_smem(256, 256));
     if (e == cudaSuccess) e = set_smem_attrs(k_score_stream<true>, kScoreStreamSmemMax);
     if (e == cudaSuccess) e = set_smem_attrs(k_score_stream<false>, kScoreStreamSmemMax);
+    if (e == cudaSuccess) e = set_smem_attrs(k_score_bulk<true>, kScoreSlabBytes);
+    if (e == cudaSuccess) e = set_smem_attrs(k_score_bulk<false>, kScoreSlabBytes);
     return e;
 }
 
@@ -548,6 +650,23 @@ cudaError_t launch_score(const lsa_dims& d, const SeqTable& tab, int max_n, cons
     }
     const int es = d.emb_dtype == LSA_BF16 ? 2 : 4;
     const int P = d.E * es / 16;
+    if (d.Q == 1 && P <= 32) {
+        // TMA-staged slabs of at most kScoreSlabBytes, at least two per SM when the rows allow
+        const int row_bytes = d.E * es;
+        const int total_rows = tab.chunk_off[d.B];
+        int rpc = kScoreSlabBytes / row_bytes;
+        const int spread = (total_rows + 2 * num_sms - 1) / (2 * num_sms);
+        if (spread < rpc) rpc = spread;
+        if (rpc < 1) rpc = 1;
+        cfg.gridDim = dim3((max_n + rpc - 1) / rpc, d.B, 1);
+        cfg.blockDim = dim3(kScoreThreads, 1, 1);
+        cfg.dynamicSmemBytes = (size_t)rpc * row_bytes;
+        if (d.emb_dtype == LSA_BF16)
+            return cudaLaunchKernelEx(&cfg, k_score_bulk<true>, (const uint8_t*)q_emb, (const uint8_t*)chunk_emb,
+                                      scores, tab, d.E, rpc, err);
+        return cudaLaunchKernelEx(&cfg, k_score_bulk<false>, (const uint8_t*)q_emb, (const uint8_t*)chunk_emb,
+                                  scores, tab, d.E, rpc, err);
+    }
     const int LPR = P < 32 ? P : 32;
     const int rows_step = (kScoreThreads / 32) * (32 / LPR) * kScoreUnroll;
     int total_rows = tab.chunk_off[d.B];
