@@ -101,8 +101,9 @@ LSA_API const char *lsa_status_string(lsa_status s);
  * device (it depends on the SM count). Writes *bytes; no launch. */
 LSA_API lsa_status lsa_workspace_size(const lsa_dims *dims, size_t *bytes);
 
-/* Clear the workspace's sticky error word (cudaMemsetAsync of its header).
- * Call once after allocating a workspace. */
+/* Clear the workspace header (cudaMemsetAsync of its first 256 bytes): the sticky
+ * error word and the arrival counters of the one-launch step, which every such step
+ * leaves at zero again. Call once after allocating a workspace. */
 LSA_API lsa_status lsa_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
 /* Chunk relevance [R3-2.2, ABS, R3-2.3 step 4].
@@ -175,7 +176,11 @@ LSA_API lsa_status lsa_sparse_decode_attn(const lsa_dims *dims, const void *q, c
 /* The fused step: score -> top-k -> attention over the kept chunks, reading K/V
  * through the kept ids (no resident copy is materialised) [R3-2.3 steps 4-7].
  * Arguments as above; chunk_ids_out [sum k_b] receives the kept ids; the scores
- * live in the workspace. Four kernels chained with programmatic dependent launch. */
+ * live in the workspace. Four kernels chained with programmatic dependent launch;
+ * small problems (Q == 1, B*H <= 48, N_b <= 256, embedding rows <= 512 bytes, kept
+ * K/V <= 16 MiB) run all four steps in one launch instead, whose arrival counters
+ * live in the workspace header: the workspace must have been initialised with
+ * lsa_workspace_init, and calls sharing a workspace must not overlap on the GPU. */
 LSA_API lsa_status lsa_decode_step(const lsa_dims *dims, const void *q_emb, const void *chunk_emb,
                            const void *q, const void *K, const void *V,
                            int32_t *chunk_ids_out, float *out, float *lse,

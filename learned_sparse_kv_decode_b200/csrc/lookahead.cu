@@ -813,14 +813,17 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     }
 }
 
-// Merge of the partials of the runs split across CTAs (log-sum-exp rule). grid (B*H, ceil(Qw/8)),
-// 256 threads: warp w merges window query blockIdx.y*8 + w; lane k owns output columns 4k..4k+3.
-__global__ void __launch_bounds__(256)
+// Merge of the partials of the runs split across CTAs (log-sum-exp rule). grid (B*H, ceil(Qw/4)),
+// 128 threads: warp w merges window query blockIdx.y*4 + w; lane k owns output columns 4k..4k+3.
+// 128-thread CTAs fit on an SM beside a k_attn_la CTA (registers), so they are resident and
+// waiting when the attention grid completes.
+constexpr int kLaMergeWarps = 4;
+__global__ void __launch_bounds__(kLaMergeWarps * 32)
 k_attn_la_merge(const float* __restrict__ part_o, const float* __restrict__ part_ml, float* __restrict__ out,
                 float* __restrict__ lse, const SeqTable tab, const LaParams lp) {
     const int g = blockIdx.x, b = g / lp.H, h = g - b * lp.H;
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int q = blockIdx.y * 8 + w;
+    const int q = blockIdx.y * kLaMergeWarps + w;
     pdl_trigger();  // the next kernel may set itself up; its reads wait for this grid
     pdl_wait();
     if (q >= lp.Qw) return;
@@ -1030,8 +1033,8 @@ cudaError_t launch_attention_la(const lsa_dims& d, const SeqTable& tab, int max_
     mc.stream = stream;
     mc.attrs = attr;
     mc.numAttrs = 1;
-    mc.gridDim = dim3(d.B * d.H, (d.Q + 7) / 8, 1);
-    mc.blockDim = dim3(256, 1, 1);
+    mc.gridDim = dim3(d.B * d.H, (d.Q + kLaMergeWarps - 1) / kLaMergeWarps, 1);
+    mc.blockDim = dim3(kLaMergeWarps * 32, 1, 1);
     mc.dynamicSmemBytes = 0;
     const float* cpo = part_o;
     const float* cpm = part_ml;

@@ -22,6 +22,11 @@ cudaError_t launch_gather(const lsa_dims& d, const SeqTable& tab, const void* K,
                           const int32_t* ids, void* K_res, void* V_res, uint32_t* err,
                           cudaStream_t stream);
 cudaError_t attn_ctas_per_device(lsa_dtype kv, int num_sms, int* out);
+bool small_step_eligible(const lsa_dims& d, int max_n, int64_t total_kept);
+size_t small_step_part_bytes(const lsa_dims& d, int64_t total_kept);
+cudaError_t launch_small_step(const lsa_dims& d, const SeqTable& tab, const void* q_emb, const void* chunk_emb,
+                              const void* q, const void* K, const void* V, int32_t* ids, float* out, float* lse,
+                              float* part, uint32_t* ws, cudaStream_t stream);
 cudaError_t score_init_attrs();
 cudaError_t topk_init_attrs();
 cudaError_t refresh_init_attrs();
@@ -162,14 +167,14 @@ lsa_status prepare(const lsa_dims* d, Prepared* p) {
 }
 
 struct WsLayout {
-    size_t scores, part_o, part_ml, ids, copy_src, copy_dst, copy_count, la_o, la_ml, total;
+    size_t scores, part_o, part_ml, ids, copy_src, copy_dst, copy_count, la_o, la_ml, small, total;
 };
 
 // The lookahead-window attention runs for bf16 K/V and windows of up to 64 queries.
 bool la_shape(const lsa_dims* d) { return d->kv_dtype == LSA_BF16 && d->Q <= la_max_queries(); }
 
-// Workspace: header (sticky error word) | scores | split partials | refresh buffers |
-// lookahead partials.
+// Workspace: header (sticky error word; arrival counters of the one-launch step) | scores |
+// split partials | refresh buffers | lookahead partials | one-launch step partials.
 WsLayout ws_layout(const lsa_dims* d, const Prepared& p, const DeviceInfo& di) {
     WsLayout w;
     const int slots = di.attn_ctas[d->kv_dtype] + d->B;
@@ -184,7 +189,10 @@ WsLayout ws_layout(const lsa_dims* d, const Prepared& p, const DeviceInfo& di) {
     const size_t la_slots = la_shape(d) ? (size_t)2 * di.la_ctas : 0;
     w.la_o = align256(w.copy_count + (size_t)d->B * 4);
     w.la_ml = align256(w.la_o + la_slots * d->Q * LSA_HEAD_DIM * 4);
-    w.total = align256(w.la_ml + la_slots * d->Q * 2 * 4);
+    // partials of the one-launch step (small problems only)
+    w.small = align256(w.la_ml + la_slots * d->Q * 2 * 4);
+    const size_t small_bytes = small_step_eligible(*d, p.max_n, p.total_kept) ? small_step_part_bytes(*d, p.total_kept) : 0;
+    w.total = align256(w.small + small_bytes);
     return w;
 }
 
@@ -312,6 +320,11 @@ lsa_status lsa_decode_step(const lsa_dims* dims, const void* q_emb, const void* 
     if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LSA_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+    if (small_step_eligible(*dims, p.max_n, p.total_kept)) {
+        // a few short sequences: the whole step in one launch
+        return cuda_status(launch_small_step(*dims, p.tab, q_emb, chunk_emb, q, K, V, chunk_ids_out, out, lse,
+                                             reinterpret_cast<float*>(at(ws, w.small)), err, st));
+    }
     float* scores = reinterpret_cast<float*>(at(ws, w.scores));
     cudaError_t e = launch_score(*dims, p.tab, p.max_n, q_emb, chunk_emb, scores, err, di.sms, st, false);
     if (e != cudaSuccess) return LSA_ERR_CUDA;

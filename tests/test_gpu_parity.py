@@ -298,6 +298,29 @@ def test_decode_step_small(lsa, case):
     _check_step(dw)
 
 
+# Small problems run the whole step in one launch (k_decode_small): one query per sequence, at most
+# 48 (sequence, head) pairs, at most 256 chunks per sequence, rows <= 512 B, kept K/V <= 16 MB.
+ONE_LAUNCH_CASES = [
+    dict(B=1, N=(256,), k=(256,), E=64, H=2, C=8, emb_dtype="f32", kv_dtype="f32"),       # k = N = 256
+    dict(B=3, N=(1, 37, 256), k=(1, 5, 19), E=128, H=16, C=16, emb_dtype="bf16", kv_dtype="bf16"),
+    dict(B=2, N=(9, 20), k=(2, 3), E=256, H=2, C=1024, emb_dtype="bf16", kv_dtype="f32"),  # 1024-token chunks
+    dict(B=6, N=(64, 3, 17, 100, 8, 50), k=(8, 3, 1, 12, 8, 7), E=128, H=8, C=64, emb_dtype="f32", kv_dtype="bf16"),
+]
+
+
+@pytest.mark.parametrize("case", ONE_LAUNCH_CASES, ids=lambda c: f"B{c['B']}-C{c['C']}-{c['emb_dtype']}-{c['kv_dtype']}")
+def test_decode_step_one_launch(lsa, case):
+    w = datagen.small_workload(seed=47, **case)
+    dw = G.DeviceWorkload(w, lsa)
+    for _ in range(3):  # the arrival counters are back at zero after every call
+        dw.out.fill_(float("nan"))
+        _run_step(lsa, dw)
+        _check_step(dw)
+    a = (dw.ids.clone(), dw.out.clone(), dw.lse.clone())
+    _run_step(lsa, dw)  # deterministic whichever CTA merges
+    assert torch.equal(a[0], dw.ids) and torch.equal(a[1], dw.out) and torch.equal(a[2], dw.lse)
+
+
 def test_decode_step_max_batch(lsa):
     # LSA_MAX_BATCH sequences, ragged lengths and keep counts, in one call
     rng = np.random.default_rng(21)
