@@ -321,6 +321,29 @@ def test_decode_step_one_launch(lsa, case):
     assert torch.equal(a[0], dw.ids) and torch.equal(a[1], dw.out) and torch.equal(a[2], dw.lse)
 
 
+@pytest.mark.parametrize("small", [True, False], ids=["one-launch", "four-kernels"])
+def test_decode_step_nonfinite_reported(lsa, small):
+    # a NaN chunk embedding gives a NaN score: reported as LSA_ERR_NONFINITE, never kept, and
+    # the step still attends over valid ids only (both the one-launch and the four-kernel path)
+    N = (40, 72) if small else (300, 129)
+    w = datagen.small_workload(B=2, N=N, k=(5, 9), E=64, H=4, emb_dtype="f32", kv_dtype="f32", seed=48)
+    dw = G.DeviceWorkload(w, lsa)
+    bad_row = 7
+    dw.chunk_emb[bad_row, 3] = float("nan")
+    lsa.lsa_decode_step(dw.dims, dw.q_emb, dw.chunk_emb, dw.q, dw.K, dw.V, dw.ids, dw.out, dw.lse, dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_ERR_NONFINITE
+    got = dw.ids.cpu().numpy()
+    koff = w.k_offsets
+    for b in range(w.B):
+        mine = got[koff[b]:koff[b + 1]]
+        assert np.all(np.diff(mine) > 0) and mine.min() >= 0 and mine.max() < w.N[b]
+        if b == 0:
+            assert bad_row not in mine
+        ref_o, _ = G.oracle_attention(dw, b, mine)
+        np.testing.assert_allclose(dw.out[b].cpu().numpy(), ref_o, rtol=0, atol=1e-4)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_OK  # the word was cleared
+
+
 def test_decode_step_max_batch(lsa):
     # LSA_MAX_BATCH sequences, ragged lengths and keep counts, in one call
     rng = np.random.default_rng(21)
