@@ -299,12 +299,16 @@ def test_decode_step_small(lsa, case):
 
 
 # Small problems run the whole step in one launch (k_decode_small): one query per sequence, at most
-# 48 (sequence, head) pairs, at most 256 chunks per sequence, rows <= 512 B, kept K/V <= 16 MB.
+# 48 (sequence, head) pairs, at most 256 chunks per sequence, rows <= 512 B, kept K/V <= 16 MB;
+# with k_b <= 8 everywhere the partials are merged inside a cluster, otherwise through the workspace.
 ONE_LAUNCH_CASES = [
     dict(B=1, N=(256,), k=(256,), E=64, H=2, C=8, emb_dtype="f32", kv_dtype="f32"),       # k = N = 256
     dict(B=3, N=(1, 37, 256), k=(1, 5, 19), E=128, H=16, C=16, emb_dtype="bf16", kv_dtype="bf16"),
     dict(B=2, N=(9, 20), k=(2, 3), E=256, H=2, C=1024, emb_dtype="bf16", kv_dtype="f32"),  # 1024-token chunks
     dict(B=6, N=(64, 3, 17, 100, 8, 50), k=(8, 3, 1, 12, 8, 7), E=128, H=8, C=64, emb_dtype="f32", kv_dtype="bf16"),
+    # k_b <= 8 everywhere: the CTAs of a (sequence, head) merge inside a thread-block cluster
+    dict(B=5, N=(8, 1, 30, 64, 3), k=(8, 1, 2, 5, 3), E=64, H=4, C=32, emb_dtype="bf16", kv_dtype="bf16"),
+    dict(B=3, N=(200, 9, 40), k=(7, 8, 1), E=128, H=8, C=128, emb_dtype="f32", kv_dtype="f32"),
 ]
 
 
