@@ -601,31 +601,32 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                         }
                     }
                 }
-                // 1. the scores of tile i, 64 columns at a time; read twice from TMEM (once for the
-                // tile max, once for P) to keep fewer registers live
+                // 1. the scores of tile i: both 64-column halves in one TMEM round trip (the softmax
+                // latency keeps the tile's V stage occupied, so it is on the ring's critical path)
                 dead = la_wait_warp(dead, sf0 + 8 * (uint32_t)(i % kSBufs), (uint32_t)(i / kSBufs) & 1u, err,
                                     &s_abort);
                 la_fence_after();
                 const uint32_t sbuf = lane_t + (uint32_t)(i % kSBufs) * kTile;
+                uint32_t sr[2][32];
+                if (!dead) {
+                    la_ld256x8(sbuf, sr[0]);
+                    la_ld256x8(sbuf + 64u, sr[1]);
+                    la_wait_ld();
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) sr[0][j] = sr[1][j] = 0u;
+                }
                 float mt0 = -INFINITY, mt1 = -INFINITY;
 #pragma unroll
                 for (int w = 0; w < 2; ++w) {
-                    uint32_t sr[32];
-                    if (!dead) {
-                        la_ld256x8(sbuf + (uint32_t)(w * 64), sr);
-                        la_wait_ld();
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) sr[j] = 0u;
-                    }
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int bit = 2 * (8 * w + j);
                         const bool v0 = (vm >> bit) & 1u, v1 = (vm >> (bit + 1)) & 1u;
-                        mt0 = fmaxf(mt0, fmaxf(v0 ? __uint_as_float(sr[4 * j]) : -INFINITY,
-                                               v1 ? __uint_as_float(sr[4 * j + 1]) : -INFINITY));
-                        mt1 = fmaxf(mt1, fmaxf(v0 ? __uint_as_float(sr[4 * j + 2]) : -INFINITY,
-                                               v1 ? __uint_as_float(sr[4 * j + 3]) : -INFINITY));
+                        mt0 = fmaxf(mt0, fmaxf(v0 ? __uint_as_float(sr[w][4 * j]) : -INFINITY,
+                                               v1 ? __uint_as_float(sr[w][4 * j + 1]) : -INFINITY));
+                        mt1 = fmaxf(mt1, fmaxf(v0 ? __uint_as_float(sr[w][4 * j + 2]) : -INFINITY,
+                                               v1 ? __uint_as_float(sr[w][4 * j + 3]) : -INFINITY));
                     }
                 }
                 mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, 1));
@@ -681,30 +682,22 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     l1 *= a1;
                 }
                 // 3. P = 2^(s c - m) as bf16 pairs over the first 64 columns of this S buffer: the
-                // pair of tokens 64w + 8j + 2cq + {0, 1} goes to column 32w + 4j + cq, whose scores
-                // (tokens 64w' with w' <= w) have all been read already. l sums the fp32 weights.
+                // pair of tokens 64w + 8j + 2cq + {0, 1} goes to column 32w + 4j + cq (the scores are
+                // all in registers already). l sums the fp32 weights.
                 const float nm0 = m0 == -INFINITY ? 0.f : -m0;  // all masked so far: every p is 0
                 const float nm1 = m1 == -INFINITY ? 0.f : -m1;
                 float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
                 for (int w = 0; w < 2; ++w) {
-                    uint32_t sr[32];
-                    if (!dead) {
-                        la_ld256x8(sbuf + (uint32_t)(w * 64), sr);
-                        la_wait_ld();
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) sr[j] = 0u;
-                    }
                     uint32_t pk[16];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int bit = 2 * (8 * w + j);
                         const bool v0 = (vm >> bit) & 1u, v1 = (vm >> (bit + 1)) & 1u;
-                        const float p00 = v0 ? la_ex2(fmaf(__uint_as_float(sr[4 * j]), lp.qscale, nm0)) : 0.f;
-                        const float p01 = v1 ? la_ex2(fmaf(__uint_as_float(sr[4 * j + 1]), lp.qscale, nm0)) : 0.f;
-                        const float p10 = v0 ? la_ex2(fmaf(__uint_as_float(sr[4 * j + 2]), lp.qscale, nm1)) : 0.f;
-                        const float p11 = v1 ? la_ex2(fmaf(__uint_as_float(sr[4 * j + 3]), lp.qscale, nm1)) : 0.f;
+                        const float p00 = v0 ? la_ex2(fmaf(__uint_as_float(sr[w][4 * j]), lp.qscale, nm0)) : 0.f;
+                        const float p01 = v1 ? la_ex2(fmaf(__uint_as_float(sr[w][4 * j + 1]), lp.qscale, nm0)) : 0.f;
+                        const float p10 = v0 ? la_ex2(fmaf(__uint_as_float(sr[w][4 * j + 2]), lp.qscale, nm1)) : 0.f;
+                        const float p11 = v1 ? la_ex2(fmaf(__uint_as_float(sr[w][4 * j + 3]), lp.qscale, nm1)) : 0.f;
                         ps0 += p00 + p01;
                         ps1 += p10 + p11;
                         const __nv_bfloat162 h0 = __floats2bfloat162_rn(p00, p01);
