@@ -20,8 +20,9 @@
 //    in the kernel parameters.
 //  * Warp 8 (producer) streams each tile's K and V rows from the full cache, through the
 //    kept chunk ids (or from a compact resident buffer), with 3-D TMA tile loads in the
-//    128-byte-swizzled layout the MMAs read: a 3-deep K ring (a K tile is free once its S has
-//    completed) and a 3-deep V ring (free once its O has). No multicast; L2 evict-first.
+//    128-byte-swizzled layout the MMAs read: a 2-deep K ring (a K tile is free once its S has
+//    completed) and a 4-deep V ring (free only once its O has, after the tile's softmax: the
+//    longer-held operand gets the deeper ring). No multicast; L2 evict-first.
 //  * Warp 9 (one thread) issues the MMAs as their inputs arrive (polling, never blocking on
 //    one barrier while another product is ready):
 //      S  = Q . K^T    M = 64, N = 128, K = 128  bf16 -> fp32 TMEM, 2 buffers
@@ -29,7 +30,7 @@
 //    M = 64 holds the window's queries once. A tcgen05 MMA with N <= 128 takes about the same
 //    time whatever its M (64 or 128) and N, so the tile is as wide as the S product allows;
 //    M = 64 does half the multiply-adds of a 128-row product, and its 16 KiB of queries leave
-//    room for the third K stage.
+//    room for a sixth ring stage.
 //  * Warps 0-3 and 4-7 are two softmax groups that take alternate tiles. Each group has
 //    its own running max m and sum l per row (log2 domain) and its own O accumulator in
 //    TMEM, so two tiles' softmax overlap. An M = 64 accumulator keeps row m in TMEM lane
@@ -63,8 +64,8 @@ constexpr int kTile = 128;                // kept tokens per tile
 constexpr int kHalfTok = kTile / 2;       // tokens of a half tile (the bad-id mask is built 64 at a time)
 constexpr int kRows = 64;                 // MMA rows (M = 64): the window's queries
 constexpr int kQmax = 64;                 // window queries per (sequence, head)
-constexpr int kKStages = 3;               // K ring depth (a K tile is free once its S has completed)
-constexpr int kVStages = 3;               // V ring depth (a V tile is free once its O has completed)
+constexpr int kKStages = 2;               // K ring depth (a K tile is free once its S has completed)
+constexpr int kVStages = 4;               // V ring depth (a V tile is free once its O has completed)
 constexpr uint32_t kHalf = kTile * 128;   // a 64-dim half of a K or V tile: 128 rows x 128 B (16 KiB)
 constexpr uint32_t kOperand = 2 * kHalf;  // a K or V tile (32 KiB)
 
@@ -347,6 +348,7 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     __shared__ __align__(8) uint64_t bar_qf, bar_qe, bar_end;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
+    __shared__ int s_anybad;          // some kept id of this CTA's tiles is out of range
     __shared__ float2 s_ml1[kRows];  // group 1's (m, l) per row, at a run end
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -377,6 +379,7 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         mbar_init(endb, 1);
         fence_mbar_init();
         s_abort = 0;
+        s_anybad = 0;
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
@@ -563,7 +566,21 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         const uint32_t lane_t = tmem + ((uint32_t)(sp * 32) << 16);
         const uint32_t o0 = lane_t + kTmemO, o1 = o0 + kDh, o_mine = g ? o1 : o0;
         LaCursor cur = la_cursor(s0, tab, lp);
-        if (lp.indexed) pdl_wait();  // the chunk ids (read for the bad-id mask) come from the preceding kernel
+        bool anybad = false;
+        if (lp.indexed) {
+            // once per CTA: does any tile of its range hold an out-of-range id? Only then does each
+            // tile build its bad-token mask (the ids' loads would otherwise sit in every tile's path)
+            pdl_wait();  // the chunk ids come from the preceding kernel
+            for (int64_t sidx = s0 + (tid & 255); sidx < s1; sidx += 256) {
+                const LaCursor u = la_cursor(sidx, tab, lp);
+                const int u0 = u.t * kTile;
+                uint64_t bad = la_bad_tokens(u, u0, ids, tab);
+                if (u.kt - u0 > kHalfTok) bad |= la_bad_tokens(u, u0 + kHalfTok, ids, tab);
+                if (bad != 0ull) s_anybad = 1;
+            }
+            la_softmax_sync();
+            anybad = *(volatile int*)&s_anybad != 0;
+        }
         float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
         bool dead = false, run_whole = false;
         int run_idx = 0;
@@ -584,7 +601,7 @@ k_attn_la(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     const int u0 = cur.t * kTile;
                     const int rem = cur.kt - u0;
                     uint64_t bad0 = 0ull, bad1 = 0ull;
-                    if (lp.indexed) {
+                    if (anybad) {
                         bad0 = la_bad_tokens(cur, u0, ids, tab);
                         if (rem > kHalfTok) bad1 = la_bad_tokens(cur, u0 + kHalfTok, ids, tab);
                     }
