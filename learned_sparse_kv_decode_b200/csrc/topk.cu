@@ -10,10 +10,12 @@
 // the lowest-index keys == T and writes the kept indices in ascending order.
 //
 // One sequence runs on a thread-block cluster of CS CTAs (CS = 1..8): CTA r owns
-// a contiguous slice of the sequence's keys (cached in its shared memory). Each
-// pass builds per-CTA digit histograms that every CTA then sums through
-// distributed shared memory (DSMEM); the ordered write uses per-CTA counts
-// exchanged the same way. Cluster barriers are hardware barriers.
+// a contiguous slice of the sequence's keys. Each pass builds per-CTA digit
+// histograms that are summed across the cluster through distributed shared memory
+// (DSMEM); the ordered write uses per-CTA counts exchanged the same way. Cluster
+// barriers are hardware barriers. Two kernels: k_topk_reg (keys in registers, up to
+// 4096 per CTA: every workload here) and k_topk (keys in shared or global memory,
+// for longer sequences).
 #include "lsa_device.cuh"
 
 namespace lsa {
@@ -319,10 +321,18 @@ k_topk(const float* __restrict__ scores, int32_t* __restrict__ ids, const SeqTab
 }
 
 // ------------------------------------------------------------------ register-resident variant
-// Each of the kTopkRegThreads threads keeps a contiguous run of R keys of its CTA's slice in registers,
-// so the four digit passes and the ordered write need one block barrier each: the digit
-// search runs redundantly in every warp, histograms are triple-buffered (the buffer a pass
-// clears was last read two passes earlier), and the write uses one block-wide scan.
+// Each of the kTopkRegThreads threads keeps a contiguous run of R keys of its CTA's slice in
+// registers, so each digit pass and the ordered write need one block barrier: the digit search
+// runs redundantly in every warp and histograms are triple-buffered (the buffer a pass clears was
+// last read two passes earlier). The keys arrive through a padded shared-memory transpose, so the
+// global loads are coalesced while each thread still owns a contiguous run. The passes stop early
+// once the bin holding the k-th key is kept whole (its count equals the keys still needed): the
+// keep set is then every key >= the bin's lower edge, with no tie to break. The ordered write
+// scans the two per-thread counts (kept outright, equal to T) packed into one word.
+// In a cluster every exchange is a push: each CTA adds its histogram into every CTA's copy of
+// the totals (remote red.add) and stores its counts into every CTA's table before the cluster
+// barrier, so that after the barrier all reads are local and no CTA waits on a trailing barrier
+// before it exits. The first barrier's arrive is issued before the loads and its wait after them.
 #ifndef LSA_TOPK_HIST
 #define LSA_TOPK_HIST 1  // histogram update: 0 = warp-aggregated (match.any), 1 = one atomic per key (faster)
 #endif
@@ -333,9 +343,9 @@ constexpr int kTopkRegThreads = LSA_TOPK_REG_THREADS;
 constexpr int kTopkRegWarps = kTopkRegThreads / 32;
 
 // Finds the digit d (of 256) where the keys above d number < need <= keys at or above d.
-// Every lane of the calling warp returns the same (digit, keys above d).
+// Every lane of the calling warp returns the same (digit, keys above d, keys in bin d).
 __device__ __forceinline__ void find_digit(const uint32_t* h256, uint32_t need, int lane,
-                                           uint32_t& digit, uint32_t& above_out) {
+                                           uint32_t& digit, uint32_t& above_out, uint32_t& bin_out) {
     uint32_t h[8], sum = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -349,12 +359,13 @@ __device__ __forceinline__ void find_digit(const uint32_t* h256, uint32_t need, 
         if (lane >= off) incl += v;
     }
     uint32_t above = incl - sum;
-    uint32_t found = 0xFFFFFFFFu, fa = 0;
+    uint32_t found = 0xFFFFFFFFu, fa = 0, fb = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         if (found == 0xFFFFFFFFu && above < need && need <= above + h[i]) {
             found = (uint32_t)(255 - 8 * lane - i);
             fa = above;
+            fb = h[i];
         }
         above += h[i];
     }
@@ -362,18 +373,46 @@ __device__ __forceinline__ void find_digit(const uint32_t* h256, uint32_t need, 
     const int src = __ffs(who) - 1;  // exactly one lane holds the digit
     digit = __shfl_sync(0xffffffffu, found, src);
     above_out = __shfl_sync(0xffffffffu, fa, src);
+    bin_out = __shfl_sync(0xffffffffu, fb, src);
 }
 
+// Add v to the u32 at the same shared-memory offset as `p` in CTA `rank` of this cluster.
+__device__ __forceinline__ void dsmem_red_add(uint32_t* p, uint32_t rank, uint32_t v) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(p)), "r"(rank));
+    asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" :: "r"(remote), "r"(v) : "memory");
+}
+// Store v to the u32 at the same shared-memory offset as `p` in CTA `rank` of this cluster.
+__device__ __forceinline__ void dsmem_st(uint32_t* p, uint32_t rank, uint32_t v) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(p)), "r"(rank));
+    asm volatile("st.shared::cluster.u32 [%0], %1;" :: "r"(remote), "r"(v) : "memory");
+}
+// The two halves of a cluster barrier, for work between the arrive and the wait.
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Shared-memory slot of slice index i in the load transpose: one pad word per 32 keeps both the
+// coalesced writes (consecutive i) and the per-thread run reads (i = R * tid + j) conflict-free
+// for R = 1, 2, 4, 8, 16.
+__device__ __forceinline__ int topk_stage_slot(int i) { return i + (i >> 5); }
+
 // grid (CS, B) with cluster (CS, 1, 1), kTopkRegThreads threads; a CTA's slice has at most
-// kTopkRegThreads * R keys.
+// kTopkRegThreads * R keys. Counts are packed 16 + 16 bits, so a sequence has at most 65535 keys.
 template <int R>
 __global__ void __launch_bounds__(kTopkRegThreads)
 k_topk_reg(const float* __restrict__ scores, int32_t* __restrict__ ids, const SeqTable tab,
            uint32_t* err, const ThresholdArgs th) {
+    constexpr int kSlice = kTopkRegThreads * R;
     __shared__ uint32_t hist[3][256];
-    __shared__ uint32_t tot[256];
-    __shared__ uint32_t w_gt[kTopkRegWarps], w_eq[kTopkRegWarps];
-    __shared__ uint32_t c_gt, c_eq;  // this CTA's totals of keys > T and == T (read by the cluster)
+    __shared__ uint32_t tot[2][256];  // cluster totals: every CTA adds its histogram into each CTA's copy
+    __shared__ uint32_t stage[kSlice + kSlice / 32];
+    __shared__ uint32_t r_cnt[kTopkMaxCluster];  // packed counts of each CTA, stored by that CTA
+    __shared__ uint32_t w_cnt[kTopkRegWarps];
     __shared__ uint32_t s_red[kTopkRegWarps], s_cnt;
 
     const int b = blockIdx.y;
@@ -392,16 +431,33 @@ k_topk_reg(const float* __restrict__ scores, int32_t* __restrict__ ids, const Se
     if (tid < 256) {
         hist[0][tid] = 0;
         hist[1][tid] = 0;
+        tot[0][tid] = 0;
+        tot[1][tid] = 0;
     }
+    if (cs > 1) cluster_arrive_release();  // every CTA running, its totals zeroed (waited below)
     pdl_wait();  // scores come from the preceding kernel
     pdl_trigger();
 
-    uint32_t kr[R];
     bool bad = false;
+    {
+        float v[R];  // every load in flight before the first store
 #pragma unroll
-    for (int j = 0; j < R; ++j) kr[j] = base + j < m ? score_key(s[base + j], bad) : 0u;
+        for (int j = 0; j < R; ++j) {
+            const int i = j * kTopkRegThreads + tid;
+            v[j] = i < m ? s[i] : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < R; ++j) {
+            const int i = j * kTopkRegThreads + tid;
+            stage[topk_stage_slot(i)] = i < m ? score_key(v[j], bad) : 0u;
+        }
+    }
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(err, kErrNonFinite);
     __syncthreads();
+    uint32_t kr[R];
+#pragma unroll
+    for (int j = 0; j < R; ++j) kr[j] = stage[topk_stage_slot(base + j)];
+    if (cs > 1) cluster_wait_acquire();
 
     if (th.enabled) {
         bool dummy = false;
@@ -412,8 +468,13 @@ k_topk_reg(const float* __restrict__ scores, int32_t* __restrict__ ids, const Se
         const int total = (int)cluster_sum<kTopkRegWarps>(c, s_red, &s_cnt, cs);
         k = max(min(total, kcap), min(th.k_min, kcap));
     }
+    // T = prefix: the k-th largest key, of which `need` are kept (lowest index first); with
+    // `whole`, prefix is the lower edge of a bin kept whole and every key >= prefix is kept.
     uint32_t prefix = 0, need = (uint32_t)k;
+    bool whole = false;
+#pragma unroll
     for (int pass = 0; pass < 4; ++pass) {
+        if (whole) break;
         const int shift = 24 - 8 * pass;
         const uint32_t himask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
         uint32_t* hp = hist[pass % 3];
@@ -430,86 +491,64 @@ k_topk_reg(const float* __restrict__ scores, int32_t* __restrict__ ids, const Se
         }
         if (tid < 256) hist[(pass + 1) % 3][tid] = 0;  // used next pass; last read two passes ago
         const uint32_t* h = hp;
-        if (cs > 1) {
-            cluster_sync_all();
-            if (tid < 256) {
-                uint32_t v[kTopkMaxCluster];
-#pragma unroll
-                for (int r = 0; r < kTopkMaxCluster; ++r) v[r] = (uint32_t)r < cs ? dsmem_ld(&hp[tid], r) : 0u;
-                uint32_t t = 0;
-#pragma unroll
-                for (int r = 0; r < kTopkMaxCluster; ++r) t += v[r];
-                tot[tid] = t;
-            }
-            h = tot;
-        }
         __syncthreads();
-        uint32_t digit, above;
-        find_digit(h, need, lane, digit, above);
+        if (cs > 1) {
+            // tot[(pass + 1) % 2] was read last pass (every warp is past the barrier above); the
+            // other CTAs add into it next pass, after the cluster barrier below
+            if (tid < 256) {
+                tot[(pass + 1) % 2][tid] = 0;
+                const uint32_t v = hp[tid];
+                if (v) {
+                    for (uint32_t r = 0; r < cs; ++r) dsmem_red_add(&tot[pass % 2][tid], r, v);
+                }
+            }
+            cluster_sync_all();
+            h = tot[pass % 2];
+        }
+        uint32_t digit, above, inbin;
+        find_digit(h, need, lane, digit, above, inbin);
         prefix |= digit << shift;
         need -= above;
-        if (cs > 1) __syncthreads();  // tot is rewritten by the next pass
+        whole = need == inbin;  // the same decision in every thread of the cluster
     }
-    const uint32_t T = prefix;  // the k-th largest key; keep `need` of the keys equal to T
+    // Kept outright: key >= T_lo, where T_lo = T + 1, or T itself when its bin is kept whole
+    // (no key maps above +inf's 0xFF800000, so T + 1 does not wrap). Keys == T that are not kept
+    // outright are tie candidates.
+    const uint32_t T = prefix, T_lo = whole ? prefix : prefix + 1u;
 
-    // ---- counts in index order: this thread's run, then a block-wide exclusive scan
-    uint32_t g = 0, e = 0;
+    // ---- packed counts in index order: low half keys kept outright, high half tie candidates
+    uint32_t c = 0;
 #pragma unroll
     for (int j = 0; j < R; ++j) {
-        if (base + j < m) {
-            g += kr[j] > T;
-            e += kr[j] == T;
-        }
+        if (base + j < m) c += kr[j] >= T_lo ? 1u : (kr[j] == T ? 0x10000u : 0u);
     }
-    uint32_t ig = g, ie = e;
+    uint32_t ic = c;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t vg = __shfl_up_sync(0xffffffffu, ig, off);
-        const uint32_t ve = __shfl_up_sync(0xffffffffu, ie, off);
-        if (lane >= off) {
-            ig += vg;
-            ie += ve;
-        }
+        const uint32_t v = __shfl_up_sync(0xffffffffu, ic, off);
+        if (lane >= off) ic += v;
     }
-    if (lane == 31) {
-        w_gt[warp] = ig;
-        w_eq[warp] = ie;
-    }
+    if (lane == 31) w_cnt[warp] = ic;
     __syncthreads();
-    uint32_t before_g = ig - g, before_e = ie - e, cta_g = 0, cta_e = 0;
+    uint32_t before = ic - c, cta = 0;
 #pragma unroll
     for (int w = 0; w < kTopkRegWarps; ++w) {
-        const uint32_t a = w_gt[w], c = w_eq[w];
-        if (w < warp) {
-            before_g += a;
-            before_e += c;
-        }
-        cta_g += a;
-        cta_e += c;
+        const uint32_t a = w_cnt[w];
+        if (w < warp) before += a;
+        cta += a;
     }
     if (cs > 1) {
-        if (tid == 0) {
-            c_gt = cta_g;
-            c_eq = cta_e;
-        }
+        if ((uint32_t)tid < cs) dsmem_st(&r_cnt[rank], (uint32_t)tid, cta);
         cluster_sync_all();
-        uint32_t vg[kTopkMaxCluster], ve[kTopkMaxCluster];
 #pragma unroll
-        for (int r = 0; r < kTopkMaxCluster; ++r) {
-            vg[r] = (uint32_t)r < rank ? dsmem_ld(&c_gt, r) : 0u;
-            ve[r] = (uint32_t)r < rank ? dsmem_ld(&c_eq, r) : 0u;
-        }
-#pragma unroll
-        for (int r = 0; r < kTopkMaxCluster; ++r) {
-            before_g += vg[r];
-            before_e += ve[r];
-        }
+        for (int r = 0; r < kTopkMaxCluster; ++r) before += (uint32_t)r < rank ? r_cnt[r] : 0u;
     }
-    // ---- ordered write: every key > T, and the lowest-index `need` keys == T
+    // ---- ordered write: every key kept outright, and the lowest-index `need` keys == T
+    uint32_t before_g = before & 0xFFFFu, before_e = before >> 16;
 #pragma unroll
     for (int j = 0; j < R; ++j) {
         if (base + j < m) {
-            if (kr[j] > T) {
+            if (kr[j] >= T_lo) {
                 const uint32_t pos = before_g + min(before_e, need);
                 if (pos < (uint32_t)k) out[pos] = lo + base + j;
                 ++before_g;
@@ -527,7 +566,6 @@ k_topk_reg(const float* __restrict__ scores, int32_t* __restrict__ ids, const Se
             out[pos] = -1;
         if (rank == 0 && tid == 0) th.counts[b] = k;
     }
-    if (cs > 1) cluster_sync_all();  // keep c_gt / c_eq alive until every CTA has read them
 }
 
 // Raise the dynamic shared-memory limit of the top-k kernel (once per device).
