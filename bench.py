@@ -552,6 +552,7 @@ def run_ours(args):
             torch.cuda.synchronize()
             torch.cuda.empty_cache()
     clk = clocks.stop()
+    read_gbs = read_stream_gbs(lsa, world)
 
     st = lsa.lsa_get_device_status(head.ws)
     if st != lsa.LSA_OK:
@@ -607,7 +608,11 @@ def run_ours(args):
                 "frac": attn_gbs / peak,
                 "frac_of_spec_8tbs": attn_gbs / SPEC_HBM_GBS,
                 "peak_note": ("peak = the measured copy bandwidth (read + write); a read-only stream can "
-                              "exceed it, so frac_of_spec_8tbs is given beside it"),
+                              "exceed it, so frac_of_spec_8tbs and frac_of_read_stream are given beside it"),
+                "read_stream_gbs": read_gbs,
+                "frac_of_read_stream": attn_gbs / read_gbs,
+                "read_stream_note": ("lsa_read_stream over 4 GiB (16-byte non-coherent loads, two 1024-thread "
+                                     "CTAs per SM), timed live in this run: the plain read ceiling"),
                 "traffic": recorded_traffic(args.workload),
                 "algorithmic_bytes_per_launch": head.attn_bytes(),
                 "launch_ms": hr["attn_ms"],
@@ -627,6 +632,17 @@ def run_ours(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def read_stream_gbs(lsa, world: int, nbytes: int = 4 << 30) -> float:
+    """GB/s of a plain DRAM read stream: lsa_read_stream over a buffer far larger than L2, 3 untimed
+    and 10 timed calls (CUDA events, max over ranks). The ceiling of a read-only kernel."""
+    import torch
+    buf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    ms = time_loop(lambda i: lsa.lsa_read_stream(buf), 10, 3, world)
+    del buf
+    torch.cuda.empty_cache()
+    return nbytes / (ms / 10 / 1e3) / 1e9
 
 
 def graph_loop(call, n: int, K: int, W: int, world: int) -> float:

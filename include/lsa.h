@@ -344,6 +344,13 @@ LSA_API lsa_status lsa_merge_partials(int32_t G, int32_t B, int32_t H, const flo
  * return LSA_OK or the first device error (NONFINITE, BAD_ID, TIMEOUT, in that order). */
 LSA_API lsa_status lsa_get_device_status(void *ws, void *stream);
 
+/* Measurement utility, not a step of the method: read `bytes` of device memory at `buf` with
+ * 16-byte non-coherent loads and discard them (grid-stride, two 1024-thread CTAs per SM), so
+ * that a caller can time a plain DRAM read stream, the ceiling of the read-only attention
+ * stream, beside a copy benchmark. `buf` 16-byte aligned and `bytes` a multiple of 16, else
+ * LSA_ERR_INVALID_ARG with nothing launched; the caller owns the buffer. Async on `stream`. */
+LSA_API lsa_status lsa_read_stream(const void *buf, size_t bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

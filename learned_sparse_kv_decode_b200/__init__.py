@@ -20,7 +20,7 @@ from .abi import (  # noqa: E402,F401
     lsa_topk_select, lsa_sparse_decode_attn_noalloc, lsa_refresh_resident,
     lsa_threshold_select, lsa_decode_step_threshold, lsa_indexer_score_fp8, lsa_decode_step_fp8,
     LSA_ENSEMBLE_MAX, LSA_ENSEMBLE_MEAN, LSA_INDEX_DIM, lsa_sparse_decode_attn_counts, lsa_shard_candidates,
-    lsa_shard_global_select, lsa_merge_partials, lsa_workspace_init, lsa_workspace_size, string,
+    lsa_shard_global_select, lsa_merge_partials, lsa_read_stream, lsa_workspace_init, lsa_workspace_size, string,
     lsa_sparse_decode_attn_lookahead, lsa_decode_step_lookahead, lsa_lookahead_partition,
     LSA_OK, LSA_ERR_INVALID_ARG, LSA_ERR_WORKSPACE, LSA_ERR_CUDA, LSA_ERR_NONFINITE,
     LSA_ERR_TIMEOUT, LSA_ERR_UNSUPPORTED, LSA_ERR_BAD_ID, LSA_F32, LSA_BF16,

@@ -79,6 +79,7 @@ def _load():
         "lsa_shard_global_select": ([dp, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32),
                                      vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "lsa_merge_partials": ([ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, vp, vp, vp, vp, vp], ctypes.c_int),
+        "lsa_read_stream": ([vp, sz, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -281,6 +282,11 @@ def lsa_sparse_decode_attn_noalloc(dims, q, K, V, chunk_ids, out, lse, stream=No
 def lsa_get_device_status(ws, stream=None) -> int:
     """Synchronise, read and clear the sticky device error word; returns the status code."""
     return lib.lsa_get_device_status(_p(ws), _stream(stream))
+
+
+def lsa_read_stream(buf, stream=None) -> None:
+    """Read every byte of the device tensor ``buf`` and discard it (a read-bandwidth probe)."""
+    _check(lib.lsa_read_stream(_p(buf), _nbytes(buf), _stream(stream)), "lsa_read_stream")
 
 
 def alloc_workspace(dims: Dims, device=None, stream=None):

@@ -14,7 +14,7 @@ from learned_sparse_kv_decode_b200 import abi  # noqa: E402
 
 def test_exports_every_header_symbol():
     names = lsa.header_symbols()
-    assert len(names) == 23
+    assert len(names) == 24
     for n in names:
         assert hasattr(abi.lib, n), n
 
@@ -55,6 +55,12 @@ def _ws_size_status(**kw):
 ])
 def test_host_validation_rejects(kw, expect):
     assert _ws_size_status(**kw) == expect
+
+
+@pytest.mark.parametrize("ptr,nbytes", [(None, 16), (16, 0), (0x1008, 16), (0x1000, 24)])
+def test_read_stream_rejects_bad_buffers(ptr, nbytes):
+    # null, empty, not 16-byte aligned, not a multiple of 16 bytes: rejected before any CUDA call
+    assert abi.lib.lsa_read_stream(ptr, nbytes, None) == lsa.LSA_ERR_INVALID_ARG
 
 
 def test_null_arguments_rejected():

@@ -152,6 +152,18 @@ def test_topk_nonfinite_reported(lsa):
     assert lsa.lsa_get_device_status(ws) == lsa.LSA_OK  # the word was cleared
 
 
+# ------------------------------------------------------------------ read-stream utility
+def test_read_stream_runs(lsa):
+    # the measurement utility reads a buffer with a ragged tail (not a multiple of the unrolled
+    # stride) and leaves the context usable; an unaligned view is rejected on the host
+    buf = torch.empty((64 << 20) + 48, dtype=torch.uint8, device="cuda")
+    lsa.lsa_read_stream(buf)
+    torch.cuda.synchronize()
+    with pytest.raises(lsa.LsaError):
+        lsa.lsa_read_stream(buf[8:8 + 1024])
+    torch.cuda.synchronize()
+
+
 # ------------------------------------------------------------------ gather
 @pytest.mark.parametrize("kv_dtype,H,C", [("f32", 8, 64), ("bf16", 16, 64), ("bf16", 2, 32), ("f32", 1, 8)])
 def test_gather_bit_exact(lsa, kv_dtype, H, C):
