@@ -553,6 +553,11 @@ def run_ours(args):
             torch.cuda.empty_cache()
     clk = clocks.stop()
     read_gbs = read_stream_gbs(lsa, world)
+    for r in results.values():  # the window attention against the same read ceiling
+        la = r.get("lookahead")
+        if la is not None:
+            la["attn_frac_of_read_stream"] = la["attn_gbs"] / read_gbs
+            la["attn_long"]["frac_of_read_stream"] = la["attn_long"]["gbs"] / read_gbs
 
     st = lsa.lsa_get_device_status(head.ws)
     if st != lsa.LSA_OK:
