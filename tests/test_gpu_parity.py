@@ -87,8 +87,11 @@ def _tie_scores(n, seed, levels=4.0):
     return (np.round(x * levels) / levels).astype(np.float32)  # many exact ties
 
 
-@pytest.mark.parametrize("N,k", [((1,), (1,)), ((7, 64), (3, 64)), ((1000, 999), (1, 998)),
-                                 ((5000, 16384), (700, 2212)), ((60000,), (6000,)),
+@pytest.mark.parametrize("N,k", [((1,), (1,)), ((7, 64), (3, 64)), ((300, 500), (40, 499)),
+                                 ((1000, 999), (1, 998)),
+                                 ((5000, 16384), (700, 2212)),
+                                 ((30000, 17000), (4000, 2)),   # 16 keys per thread in an 8-CTA cluster
+                                 ((60000,), (6000,)),
                                  ((120_000,), (16_000,)),       # per-CTA slices in shared memory
                                  ((400_000, 3), (54_000, 2))])  # slices too big for shared memory
 def test_topk_bit_exact_with_ties(lsa, N, k):
