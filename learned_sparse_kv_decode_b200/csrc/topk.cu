@@ -4,10 +4,11 @@
 // step 5): a top-k keep mask over the chunk scores decides which chunks stay
 // resident. Ties go to the lower chunk index; -0.0 and +0.0 are equal.
 //
-// Exact radix select on order-preserving 32-bit keys, four 8-bit digit passes
+// Exact radix select on order-preserving 32-bit keys, up to four 8-bit digit passes
 // (most significant first), finding T, the k-th largest key, and how many keys
 // equal to T must be kept. A final pass in index order keeps every key > T plus
-// the lowest-index keys == T and writes the kept indices in ascending order.
+// the lowest-index keys == T and writes the kept indices in ascending order. (The
+// register kernel stops early when the bin holding the k-th key is kept whole.)
 //
 // One sequence runs on a thread-block cluster of CS CTAs (CS = 1..8): CTA r owns
 // a contiguous slice of the sequence's keys. Each pass builds per-CTA digit
