@@ -80,3 +80,14 @@ def test_valid_dims_need_a_device_here():
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert _ws_size_status() == lsa.LSA_ERR_CUDA
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    # no fallback: without the CUDA library the binding refuses to load
+    old = abi.LIB_PATH
+    abi.LIB_PATH = str(tmp_path / "liblsa_b200.so")
+    try:
+        with pytest.raises(ImportError):
+            abi._load()
+    finally:
+        abi.LIB_PATH = old
