@@ -10,7 +10,8 @@ exchanges between them are all-gathers of fixed-size tensors:
 
 `run_distributed` drives the phases with torch.distributed (NCCL over NVLink on GPUs, one
 process per GPU; the only collectives are those two all-gathers, each carried out as one
-all_gather_into_tensor per tensor). `run_emulated` drives G shard objects in one process
+all_gather_into_tensor per tensor; under a host backend such as gloo the device tensors are
+gathered through host memory). `run_emulated` drives G shard objects in one process
 (the all-gathers become stacks), which exercises every kernel of the sharded path on one
 GPU. All arithmetic happens in the library's CUDA kernels (`CudaShardBackend`); the backend
 object exists so that the exchange logic can also be checked on the host with an exact
@@ -148,6 +149,8 @@ def _all_gather(t: torch.Tensor, world: int) -> torch.Tensor:
     """[world, *t.shape] in rank order (gathered as a concatenation along dim 0, the form
     every backend accepts)."""
     import torch.distributed as dist
+    if t.is_cuda and dist.get_backend() != "nccl":  # a host collective backend (gloo): via host memory
+        return _all_gather(t.cpu(), world).to(t.device)
     t = t.contiguous()
     out = torch.empty((world * t.shape[0], *t.shape[1:]), dtype=t.dtype, device=t.device)
     dist.all_gather_into_tensor(out, t)
