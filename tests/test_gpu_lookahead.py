@@ -132,6 +132,37 @@ def test_lookahead_bad_id_reported(lsa, C):
     _free()
 
 
+def _random_window_case(seed):
+    """A random window-attention shape: ragged N_b and k_b, chunk length 8 to 256 (several chunks
+    per tile, or several tiles per chunk), a partial or full window of queries, 1 to 16 heads."""
+    rng = np.random.default_rng(3000 + seed)
+    B = int(rng.integers(1, 6))
+    C = int(rng.choice([8, 16, 32, 64, 128, 256]))
+    N = [int(rng.integers(1, 4096 // C + 2)) for _ in range(B)]
+    k = [int(rng.integers(1, n + 1)) for n in N]
+    return dict(B=B, N=tuple(N), k=tuple(k), C=C, Q=int(rng.integers(1, 65)),
+                H=int(rng.choice([1, 2, 4, 8, 16])))
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_lookahead_attention_random_shapes(lsa, seed):
+    w = datagen.small_workload(E=64, kv_dtype="bf16", emb_dtype="bf16", seed=4000 + seed,
+                               **_random_window_case(seed))
+    win = Window(w, lsa)
+    ids = win.random_ids(seed)
+    ids_d = torch.from_numpy(np.concatenate(ids)).cuda()
+    lsa.lsa_sparse_decode_attn_lookahead(win.dw.dims, win.q, win.dw.K, win.dw.V, ids_d, win.out, win.lse,
+                                         win.dw.ws)
+    assert lsa.lsa_get_device_status(win.dw.ws) == lsa.LSA_OK
+    big = w.Q * w.H * max(w.k) * w.C > 4_000_000
+    for b in range(w.B):
+        heads = sorted({0, w.H - 1}) if big else None
+        queries = sorted({0, w.Q // 2, w.Q - 1}) if big else None
+        _compare(win, b, ids[b], heads, queries)
+    del win
+    _free()
+
+
 def test_lookahead_resident_equals_indexed(lsa):
     # the same tiles in the same order: the resident form gives bit-identical results
     w = datagen.small_workload(B=2, N=(40, 72), k=(5, 9), C=16, E=64, Q=64, H=4, kv_dtype="bf16",

@@ -376,6 +376,38 @@ def test_decode_step_max_batch(lsa):
     _free()
 
 
+def _fuzz_case(seed):
+    """A random valid fused-step shape: ragged N_b and k_b, dtypes, heads, chunk length, queries
+    (Q = 1 takes the CUDA-core scorer or, when small, the one-launch step; Q > 1 with bf16
+    embeddings the tensor-core scorer), with the full K/V cache kept under 512 MB."""
+    rng = np.random.default_rng(1000 + seed)
+    while True:
+        B = int(rng.integers(1, 7))
+        emb_dtype = str(rng.choice(["f32", "bf16"]))
+        kv_dtype = str(rng.choice(["f32", "bf16"]))
+        E = int(rng.choice([64, 128] if emb_dtype == "f32" else [64, 128, 256]))
+        Q = int(rng.choice([1, 1, 3, 64])) if emb_dtype == "bf16" else int(rng.choice([1, 1, 3]))
+        H = int(rng.choice([1, 2, 4, 8, 16, 32]))
+        C = int(rng.choice([8, 16, 32, 64, 128]))
+        N = [int(rng.integers(1, 260)) for _ in range(B)]
+        k = [int(rng.integers(1, min(n, 70) + 1)) for n in N]
+        kv_bytes = sum(N) * C * H * 128 * (2 if kv_dtype == "bf16" else 4) * 2
+        if kv_bytes <= (512 << 20):
+            return dict(B=B, N=tuple(N), k=tuple(k), E=E, Q=Q, H=H, C=C, emb_dtype=emb_dtype,
+                        kv_dtype=kv_dtype, seed=2000 + seed)
+
+
+@pytest.mark.parametrize("seed", range(48))
+def test_decode_step_random_shapes(lsa, seed):
+    # every sequence and head against the oracle: ids (near-tie rule) and attention on them
+    w = datagen.small_workload(**_fuzz_case(seed))
+    dw = G.DeviceWorkload(w, lsa)
+    _run_step(lsa, dw)
+    _check_step(dw)
+    del dw
+    _free()
+
+
 def test_decode_step_deterministic(lsa):
     w = datagen.small_workload(B=2, N=(300, 129), k=(40, 7), E=128, H=16, emb_dtype="bf16", kv_dtype="bf16")
     dw = G.DeviceWorkload(w, lsa)
