@@ -81,6 +81,63 @@ def test_score_chunks_parity(lsa, case):
         G.check_scores(got[off[b]:off[b + 1]], ref, G.score_tolerance(qf, ef))
 
 
+@pytest.mark.parametrize("seed", range(24))
+def test_score_chunks_random_shapes(lsa, seed):
+    # random ragged batches over every scorer: one query (staged stream), several queries on the
+    # CUDA cores (fp32) or on the tensor cores (bf16, E a multiple of 16), up to 256 queries
+    rng = np.random.default_rng(5000 + seed)
+    emb_dtype = str(rng.choice(["f32", "bf16"]))
+    E = int(rng.choice([16, 32, 64, 128, 256] if emb_dtype == "bf16" else [64, 128, 256]))
+    Q = int(rng.choice([1, 1, 2, 5, 16, 64, 200, 256]))
+    if emb_dtype == "f32":  # the CUDA-core scorer holds the queries in shared memory (<= 200 KiB)
+        Q = min(Q, 200 * 1024 // (4 * E))
+    B = int(rng.integers(1, 9))
+    N = tuple(int(rng.integers(1, 700)) for _ in range(B))
+    w = datagen.small_workload(B=B, N=N, E=E, Q=Q, k=[1] * B, H=4, emb_dtype=emb_dtype, seed=5100 + seed,
+                               plant="copy_query" if Q > 1 else "copy")
+    dw = G.DeviceWorkload(w, lsa, with_kv=False)
+    lsa.lsa_score_chunks(dw.dims, dw.q_emb, dw.chunk_emb, dw.scores, dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_OK
+    got = dw.scores.cpu().numpy()
+    off = w.chunk_offsets
+    for b in range(w.B):
+        qf, ef = dw.q_emb_f(b), dw.emb_f(b)
+        G.check_scores(got[off[b]:off[b + 1]], oracle.chunk_scores(qf, ef), G.score_tolerance(qf, ef))
+
+
+@pytest.mark.parametrize("seed", range(24))
+def test_topk_and_threshold_random(lsa, seed):
+    # random ragged sequences of continuous or tie-heavy scores, random k, and a random threshold
+    rng = np.random.default_rng(6000 + seed)
+    B = int(rng.integers(1, 9))
+    N = tuple(int(rng.integers(1, 40000 if seed % 4 == 0 else 3000)) for _ in range(B))
+    k = tuple(int(rng.integers(1, n + 1)) for n in N)
+    w = datagen.small_workload(B=B, N=N, k=k, E=64)
+    dims = G.dims_of(w, lsa)
+    ws = lsa.alloc_workspace(dims)
+    s = np.concatenate([_tie_scores(n, 6100 + 10 * seed + i, levels=float(rng.choice([4.0, 1e6])))
+                        for i, n in enumerate(N)])
+    sd = torch.from_numpy(s).cuda()
+    ids = torch.empty(w.total_kept, dtype=torch.int32, device="cuda")
+    lsa.lsa_topk_select(dims, sd, ids, ws)
+    assert lsa.lsa_get_device_status(ws) == lsa.LSA_OK
+    got = ids.cpu().numpy()
+    off, koff = w.chunk_offsets, w.k_offsets
+    for b in range(w.B):
+        np.testing.assert_array_equal(got[koff[b]:koff[b + 1]], oracle.topk(s[off[b]:off[b + 1]].astype(np.float64), k[b]))
+    tau = np.float32(np.quantile(s, rng.uniform(0.5, 0.99)))
+    k_min = int(rng.integers(1, 5))
+    cnt = torch.zeros(w.B, dtype=torch.int32, device="cuda")
+    lsa.lsa_threshold_select(dims, sd, tau, k_min, ids, cnt, ws)
+    assert lsa.lsa_get_device_status(ws) == lsa.LSA_OK
+    got, got_cnt = ids.cpu().numpy(), cnt.cpu().numpy()
+    for b in range(w.B):
+        ref = oracle.threshold_select(s[off[b]:off[b + 1]].astype(np.float64), tau, k_min, k[b])
+        assert got_cnt[b] == len(ref)
+        np.testing.assert_array_equal(got[koff[b]:koff[b] + len(ref)], ref)
+        assert (got[koff[b] + len(ref):koff[b + 1]] == -1).all()
+
+
 # ------------------------------------------------------------------ top-k
 def _tie_scores(n, seed, levels=4.0):
     x = datagen.normal_f32(seed, 1, np.arange(n))
