@@ -234,6 +234,32 @@ def test_decode_step_lookahead(lsa, case):
         _compare(win, b, gids)
 
 
+@pytest.mark.parametrize("seed", range(12))
+def test_decode_step_lookahead_random_shapes(lsa, seed):
+    # the fused window step over random ragged batches: kept ids, then every query and head
+    rng = np.random.default_rng(8000 + seed)
+    B = int(rng.integers(1, 5))
+    N = tuple(int(rng.integers(1, 300)) for _ in range(B))
+    k = tuple(int(rng.integers(1, min(n, 60) + 1)) for n in N)
+    case = dict(B=B, N=N, k=k, E=int(rng.choice([64, 128, 256])), Q=int(rng.integers(1, 65)),
+                H=int(rng.choice([1, 2, 4, 8, 16])), C=int(rng.choice([16, 32, 64, 128])), plant="copy_query")
+    w = datagen.small_workload(emb_dtype="bf16", kv_dtype="bf16", seed=8100 + seed, **case)
+    win = Window(w, lsa)
+    dw = win.dw
+    lsa.lsa_decode_step_lookahead(dw.dims, dw.q_emb, dw.chunk_emb, win.q, dw.K, dw.V, dw.ids, win.out, win.lse,
+                                  dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_OK
+    got = dw.ids.cpu().numpy()
+    big = w.Q * w.H * max(w.k) * w.C > 4_000_000
+    for b in range(w.B):
+        ref_s = oracle.chunk_scores(dw.q_emb_f(b), dw.emb_f(b))
+        gids = got[w.k_offsets[b]:w.k_offsets[b + 1]]
+        G.check_ids(gids, oracle.topk(ref_s, w.k[b]), ref_s, w.k[b])
+        _compare(win, b, gids, sorted({0, w.H - 1}) if big else None, sorted({0, w.Q // 2, w.Q - 1}) if big else None)
+    del win, dw
+    _free()
+
+
 def test_decode_step_lookahead_full_size_1m(lsa):
     # the 1M lookahead workload in the launch configuration the benchmark times: all kept ids,
     # sampled (head, query) outputs

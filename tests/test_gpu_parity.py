@@ -244,6 +244,34 @@ def test_gather_bit_exact(lsa, kv_dtype, H, C):
         np.testing.assert_array_equal(Vg[rows], dw.kv_f("V", b, tok))
 
 
+@pytest.mark.parametrize("seed", range(16))
+def test_gather_random_shapes(lsa, seed):
+    # random ragged batches, heads, chunk lengths and kept sets: every gathered row bit-exact
+    rng = np.random.default_rng(7000 + seed)
+    kv_dtype = str(rng.choice(["f32", "bf16"]))
+    H = int(rng.choice([1, 2, 4, 8, 16]))
+    C = int(rng.choice([8, 16, 32, 64, 128]))
+    B = int(rng.integers(1, 7))
+    N = tuple(int(rng.integers(1, 80)) for _ in range(B))
+    k = tuple(int(rng.integers(1, n + 1)) for n in N)
+    w = datagen.small_workload(B=B, N=N, k=k, E=64, H=H, C=C, kv_dtype=kv_dtype, seed=7100 + seed)
+    dw = G.DeviceWorkload(w, lsa)
+    ids = np.concatenate([np.sort(rng.permutation(n)[:kk]) for n, kk in zip(N, k)]).astype(np.int32)
+    Kr = torch.empty((w.total_kept * C, H, w.Dh), dtype=G.tdtype(kv_dtype), device="cuda")
+    Vr = torch.empty_like(Kr)
+    lsa.lsa_gather_kv(dw.dims, dw.K, dw.V, torch.from_numpy(ids).cuda(), Kr, Vr, dw.ws)
+    assert lsa.lsa_get_device_status(dw.ws) == lsa.LSA_OK
+    koff = w.k_offsets
+    Kg, Vg = Kr.float().cpu().numpy(), Vr.float().cpu().numpy()
+    for b in range(w.B):
+        tok = oracle.kept_tokens(ids[koff[b]:koff[b + 1]], C)
+        rows = slice(koff[b] * C, koff[b + 1] * C)
+        np.testing.assert_array_equal(Kg[rows], dw.kv_f("K", b, tok))
+        np.testing.assert_array_equal(Vg[rows], dw.kv_f("V", b, tok))
+    del dw
+    _free()
+
+
 def test_gather_bad_id_reported(lsa):
     w = datagen.small_workload(B=1, N=(5,), k=(2,), E=64, H=2)
     dw = G.DeviceWorkload(w, lsa)
