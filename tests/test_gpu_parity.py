@@ -559,6 +559,18 @@ REFRESH_CASES = [
 ]
 
 
+def _random_refresh_case(seed):
+    rng = np.random.default_rng(9000 + seed)
+    B = int(rng.integers(1, 6))
+    N = tuple(int(rng.integers(1, 400)) for _ in range(B))
+    dt = str(rng.choice(["f32", "bf16"]))
+    return dict(B=B, N=N, k=tuple(int(rng.integers(1, n + 1)) for n in N), E=int(rng.choice([64, 128])),
+                H=int(rng.choice([1, 2, 4, 8])), C=int(rng.choice([16, 32, 64])), kv_dtype=dt, emb_dtype=dt)
+
+
+REFRESH_CASES += [_random_refresh_case(i) for i in range(8)]  # seeded random ragged shapes
+
+
 def _check_resident(dw, slots, Kr, Vr, skip=None):
     w = dw.w
     Kg, Vg = Kr.float().cpu().numpy(), Vr.float().cpu().numpy()
