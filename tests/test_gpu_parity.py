@@ -725,6 +725,16 @@ FP8_CASES = [
 ]
 
 
+def _random_fp8_case(seed):
+    rng = np.random.default_rng(9500 + seed)
+    B = int(rng.integers(1, 6))
+    return dict(B=B, N=tuple(int(rng.integers(1, 700)) for _ in range(B)), L=int(rng.integers(1, 4)),
+                Hn=16 * int(rng.integers(1, 17)), mean=bool(rng.integers(0, 2)))
+
+
+FP8_CASES += [_random_fp8_case(i) for i in range(8)]  # seeded random shapes
+
+
 @pytest.mark.parametrize("case", FP8_CASES, ids=lambda c: f"B{c['B']}-L{c['L']}-H{c['Hn']}-{'mean' if c['mean'] else 'max'}")
 def test_indexer_score_fp8_parity(lsa, case):
     w = datagen.small_workload(B=case["B"], N=case["N"], k=[1] * case["B"], E=128, emb_dtype="bf16",
